@@ -1,0 +1,344 @@
+"""Pins for the float64 oracle, checked against things other than itself.
+
+Every check below is a closed form, a hand-derived worked value, a library
+routine (torch's float64 scaled-dot-product attention, torch's bfloat16 and
+float8_e4m3fn casts) or an invariant, chosen so that a plausible mistake in
+the oracle (a dropped term, a wrong sign, index or axis, a transposed
+operand, a wrong rounding rule) fails at least one of them.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from diffusion_transformer_joint_dit_b200 import inputs as I
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+# ----------------------------------------------------------------- bf16 ----
+
+def test_bf16_round_matches_torch_cast_on_float32_values():
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal(20000) * np.exp2(rng.integers(-20, 20, 20000))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.bf16_round(x.astype(np.float64)), ref)
+
+
+def test_bf16_round_ties_to_even():
+    # ulp(1) in bf16 is 2**-7; 1 + 2**-8 is a tie between 1 and 1 + 2**-7.
+    assert O.bf16_round(1 + 2.0 ** -8) == 1.0
+    # 1 + 1.5 * 2**-7 ties between 1 + 2**-7 (odd) and 1 + 2**-6 (even).
+    assert O.bf16_round(1 + 1.5 * 2.0 ** -7) == 1 + 2.0 ** -6
+    assert O.bf16_round(-(1 + 2.0 ** -8)) == -1.0
+
+
+def test_bf16_ulp_distance():
+    a = np.array([1.0, 1.0, -1.0, 0.0])
+    b = np.array([1.0 + 2.0 ** -7, 1.0 + 2.0 ** -6, -1.0 - 2.0 ** -7, -0.0])
+    assert list(O.bf16_ulp_distance(a, b)) == [1, 2, 1, 0]
+
+
+# -------------------------------------------------------------- RMSNorm ----
+
+def test_rmsnorm_hand_case():
+    x = np.tile([3.0, 4.0], 64)            # mean(x^2) = 12.5
+    y = O.rmsnorm(x, eps=1e-6)
+    r = math.sqrt(12.5 + 1e-6)
+    assert np.allclose(y[:2], [3 / r, 4 / r], rtol=0, atol=1e-15)
+
+
+def test_rmsnorm_unit_rms_and_scale_invariance():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((5, 128))
+    y = O.rmsnorm(x, eps=0.0)
+    assert np.allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, atol=1e-14)
+    assert np.allclose(O.rmsnorm(37.5 * x, eps=0.0), y, atol=1e-13)
+
+
+def test_rmsnorm_weight_is_channelwise():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((4, 128))
+    w = rng.uniform(0.5, 2, 128)
+    assert np.allclose(O.rmsnorm(x, w), O.rmsnorm(x) * w[None, :], atol=1e-14)
+
+
+# --------------------------------------------------------- positions ----
+
+def test_token_positions_small_grid():
+    rows, cols = O.token_positions(2, 2, 3, ref_h=2, ref_w=2, ref_row_offset=2)
+    assert list(rows) == [0, 0, 0, 0, 0, 1, 1, 1, 2, 2, 3, 3]
+    assert list(cols) == [0, 0, 0, 1, 2, 0, 1, 2, 0, 1, 0, 1]
+
+
+# ----------------------------------------------------------------- RoPE ----
+
+def _unit(ch, d=128):
+    x = np.zeros((1, 1, d))
+    x[0, 0, ch] = 1.0
+    return x
+
+
+def test_rope_identity_at_origin():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((3, 2, 128))
+    assert np.array_equal(O.rope_2d(x, np.zeros(3), np.zeros(3)), x)
+
+
+def test_rope_row_half_frequency_and_sign():
+    # pair i=16 of the row half: omega = 10000**(-32/64) = 1e-2; pos 100 -> 1 rad
+    y = O.rope_2d(_unit(32), np.array([100]), np.array([0]))
+    expect = np.zeros(128)
+    expect[32], expect[33] = math.cos(1.0), math.sin(1.0)
+    assert np.allclose(y[0, 0], expect, atol=1e-15)
+
+
+def test_rope_col_half_odd_element():
+    # pair i=8 of the column half: omega = 10000**(-16/64) = 0.1; pos 25 -> 2.5 rad
+    # (a, b) = (0, 1) rotates to (-sin, cos).
+    y = O.rope_2d(_unit(64 + 17), np.array([7]), np.array([25]))
+    expect = np.zeros(128)
+    expect[80], expect[81] = -math.sin(2.5), math.cos(2.5)
+    assert np.allclose(y[0, 0], expect, atol=1e-14)
+
+
+def test_rope_pair0_rotates_by_position_radians():
+    for pos in (1, 5, 127, 255):
+        y = O.rope_2d(_unit(0), np.array([pos]), np.array([3]))
+        assert math.isclose(y[0, 0, 0], math.cos(pos), abs_tol=1e-13)
+        assert math.isclose(y[0, 0, 1], math.sin(pos), abs_tol=1e-13)
+
+
+def test_rope_matches_complex_rotation():
+    """Independent formulation: pairs as complex numbers times e^{i phi}."""
+    rng = np.random.default_rng(5)
+    N, H, d = 6, 3, 128
+    x = rng.standard_normal((N, H, d))
+    pr, pc = rng.integers(0, 300, N), rng.integers(0, 300, N)
+    y = O.rope_2d(x, pr, pc)
+    z = x[..., 0::2] + 1j * x[..., 1::2]                      # [N, H, 64]
+    freq = np.concatenate([10000.0 ** (-np.arange(32) / 32.0)] * 2)
+    pos = np.concatenate([np.repeat(pr[:, None], 32, 1), np.repeat(pc[:, None], 32, 1)], 1)
+    zr = z * np.exp(1j * pos[:, None, :] * freq[None, None, :])
+    assert np.allclose(y[..., 0::2], zr.real, atol=1e-12)
+    assert np.allclose(y[..., 1::2], zr.imag, atol=1e-12)
+
+
+def test_rope_preserves_pair_norms_and_relative_positions():
+    rng = np.random.default_rng(6)
+    q = rng.standard_normal((1, 1, 128))
+    k = rng.standard_normal((1, 1, 128))
+    p, pp, delta = (3, 9), (40, 2), (128, 17)
+    qr = O.rope_2d(q, [p[0]], [p[1]])
+    kr = O.rope_2d(k, [pp[0]], [pp[1]])
+    qs = O.rope_2d(q, [p[0] + delta[0]], [p[1] + delta[1]])
+    ks = O.rope_2d(k, [pp[0] + delta[0]], [pp[1] + delta[1]])
+    assert math.isclose(float(np.sum(qr * kr)), float(np.sum(qs * ks)), rel_tol=1e-12, abs_tol=1e-12)
+    n0 = q[..., 0::2] ** 2 + q[..., 1::2] ** 2
+    n1 = qr[..., 0::2] ** 2 + qr[..., 1::2] ** 2
+    assert np.allclose(n0, n1, atol=1e-13)
+
+
+# ------------------------------------------------------------- prologue ----
+
+def test_prologue_norm_then_rope_hand_case():
+    """Norm first (with a non-uniform weight), RoPE second, on one token."""
+    q = np.zeros((1, 1, 1, 128))
+    q[..., 0], q[..., 1] = 3.0, 4.0            # mean(x^2) = 25/128
+    w = np.ones(128)
+    w[0] = 2.0
+    qp, kp = O.prologue(q, q, n_txt=0, img_h=1, img_w=1, q_norm_w=w, eps=0.0)
+    # image token 0 sits at (0, 0): no rotation.  Now move it to row 2 via a
+    # 3x1 grid (token index 2 -> (2, 0)).
+    q3 = np.zeros((1, 3, 1, 128))
+    q3[0, 2, 0, 0], q3[0, 2, 0, 1] = 3.0, 4.0
+    qp3, _ = O.prologue(q3, q3, n_txt=0, img_h=3, img_w=1, q_norm_w=w, eps=0.0)
+    r = math.sqrt(25.0 / 128.0)
+    a, b = 3.0 / r * 2.0, 4.0 / r             # normalised and weighted
+    assert np.allclose(qp[0, 0, 0, :2], [a, b], atol=1e-12)
+    c, s = math.cos(2.0), math.sin(2.0)
+    assert np.allclose(qp3[0, 2, 0, :2], [a * c - b * s, a * s + b * c], atol=1e-12)
+    # RoPE first then norm would give a different pair (the weight would hit
+    # the rotated value): make sure the two orders really differ here.
+    alt = O.rmsnorm(O.rope_2d(q3, [0, 1, 2], [0, 0, 0]), w, eps=0.0)[0, 2, 0, :2]
+    assert not np.allclose(alt, qp3[0, 2, 0, :2])
+
+
+def test_prologue_invariant_to_row_scaling_of_inputs():
+    """RMSNorm makes the prologue blind to per-row gains (outlier rows)."""
+    w = I.WORKLOADS["tiny"]
+    q, k, _ = I.make_qkv(w, seed=0)
+    kf = k.double().numpy()
+    k8 = kf.copy()
+    k8[0, 5, 1, :] *= 8.0
+    _, a = O.prologue(kf, kf, n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w, eps=0.0)
+    _, b = O.prologue(k8, k8, n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w, eps=0.0)
+    assert np.allclose(a, b, atol=1e-12)
+
+
+# ----------------------------------------------------------------- E4M3 ----
+
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0x08, 2.0 ** -6),
+    (0x30, 0.5), (0x38, 1.0), (0x39, 1.125), (0x40, 2.0), (0x77, 240.0),
+    (0x7E, 448.0), (0xFE, -448.0), (0xB8, -1.0),
+])
+def test_e4m3_decode_closed_form(code, value):
+    assert O.e4m3_decode(code) == value
+
+
+def test_e4m3_decode_all_codes_against_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    mine = O.e4m3_decode(codes)
+    nan = np.isnan(ref)
+    assert list(np.nonzero(nan)[0]) == [0x7F, 0xFF]
+    assert np.array_equal(np.isnan(mine), nan)
+    assert np.array_equal(mine[~nan], ref[~nan])
+
+
+def test_e4m3_encode_against_torch_cast():
+    rng = np.random.default_rng(7)
+    v = (rng.standard_normal(50000) * np.exp2(rng.integers(-12, 9, 50000))).astype(np.float32)
+    v = np.clip(v, -448, 448)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = O.e4m3_encode(v)
+    # torch keeps -0 for tiny negatives; the oracle maps them to +0 (same value)
+    same = (mine == ref) | ((O.e4m3_decode(mine) == 0) & (O.e4m3_decode(ref) == 0))
+    assert same.all()
+
+
+def test_e4m3_ties_and_saturation():
+    assert O.e4m3_encode(1.0625) == 0x38       # tie 1.0 / 1.125 -> even (1.0)
+    assert O.e4m3_encode(1.1875) == 0x3A       # tie 1.125 / 1.25 -> even (1.25)
+    assert O.e4m3_encode(3 * 2.0 ** -10) == 0x02   # subnormal tie 1 / 2 quanta -> 2
+    assert O.e4m3_encode(464.0) == 0x7E
+    assert O.e4m3_encode(1e6) == 0x7E
+    assert O.e4m3_encode(-1e6) == 0xFE
+
+
+def test_e4m3_roundtrip_all_finite_codes():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F and c != 0x80])
+    assert np.array_equal(O.e4m3_encode(O.e4m3_decode(codes)), codes)
+
+
+# ------------------------------------------------------ block quantiser ----
+
+def test_block_quant_constant_block():
+    x = np.full((1, 64, 1, 128), 2.0, dtype=np.float32)
+    codes, scales = O.block_quantize_e4m3(x)
+    assert scales[0, 0, 0] == np.float32(2.0) / np.float32(448.0)
+    assert (codes == 0x7E).all()
+
+
+def test_block_quant_absmax_448_is_identity_scale():
+    rng = np.random.default_rng(8)
+    x = np.clip(rng.standard_normal((1, 64, 1, 128)) * 100, -448, 448).astype(np.float32)
+    x[0, 3, 0, 5] = -448.0
+    codes, scales = O.block_quantize_e4m3(x)
+    assert scales[0, 0, 0] == 1.0
+    assert np.array_equal(codes, O.e4m3_encode(x))
+
+
+def test_block_quant_zero_block_and_partial_tail():
+    x = np.zeros((1, 70, 2, 128), dtype=np.float32)
+    x[0, 66, 1, 0] = 3.0                     # only in the 6-token tail block of head 1
+    codes, scales = O.block_quantize_e4m3(x)
+    assert scales.shape == (1, 2, 2)
+    assert scales[0, 0, 0] == 1.0 and scales[0, 0, 1] == 1.0 and scales[0, 1, 0] == 1.0
+    assert scales[0, 1, 1] == np.float32(3.0) / np.float32(448.0)
+    assert codes[0, 66, 1, 0] == 0x7E and codes.sum() == 0x7E
+
+
+def test_block_quant_error_bound_and_block_independence():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((2, 150, 3, 128)).astype(np.float32)
+    x[:, :, 2, :] *= 1000.0                  # a loud head must not change the others
+    codes, scales = O.block_quantize_e4m3(x)
+    deq = O.dequantize_e4m3(codes, scales)
+    s = np.repeat(scales.astype(np.float64), 64, axis=2)[:, :, :150].transpose(0, 2, 1)[..., None]
+    err = np.abs(deq - x)
+    # 3 mantissa bits: half-ulp relative bound 2**-4 (normal range), plus the
+    # subnormal quantum 2**-10 * scale; plus the float32 rounding of x * inv.
+    bound = np.abs(x) * (2.0 ** -4 + 2.0 ** -22) + s * 2.0 ** -10
+    assert (err <= bound).all()
+    c2, s2 = O.block_quantize_e4m3(x[:, :, :2, :])
+    assert np.array_equal(c2, codes[:, :, :2, :]) and np.array_equal(s2, scales[:, :2, :])
+
+
+# ------------------------------------------------------------ attention ----
+
+def test_attention_hand_two_keys():
+    q = np.array([[[[1.0]]]])                               # B=N_q=H=d=1
+    k = np.array([[[[0.0]], [[math.log(3.0)]]]]).reshape(1, 2, 1, 1)
+    v = np.array([1.0, 5.0]).reshape(1, 2, 1, 1)
+    out, lse = O.joint_attention(np.repeat(q, 2, axis=1), k, v, 1.0, rows=[0])
+    assert math.isclose(out[0, 0, 0, 0], 4.0, rel_tol=1e-14)   # 1/4*1 + 3/4*5
+    assert math.isclose(lse[0, 0, 0], math.log(4.0), rel_tol=1e-14)
+
+
+def test_attention_matches_torch_sdpa_float64():
+    rng = np.random.default_rng(10)
+    B, N, H, d = 2, 77, 3, 128
+    q, k, v = (rng.standard_normal((B, N, H, d)) for _ in range(3))
+    scale = 1 / math.sqrt(d)
+    out, lse = O.joint_attention(q, k, v, scale)
+    t = lambda a: torch.from_numpy(a).permute(0, 2, 1, 3)   # [B, H, N, d]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), scale=scale)
+    assert np.allclose(out, ref.permute(0, 2, 1, 3).numpy(), atol=1e-12)
+    s = torch.einsum("bhnd,bhmd->bhnm", t(q), t(k)) * scale
+    assert np.allclose(lse, torch.logsumexp(s, dim=-1).numpy(), atol=1e-12)
+
+
+def test_attention_invariants():
+    rng = np.random.default_rng(11)
+    B, N, H, d = 1, 40, 2, 128
+    q, k, v = (rng.standard_normal((B, N, H, d)) for _ in range(3))
+    # rows of softmax sum to 1: V of ones gives ones
+    out, _ = O.joint_attention(q, k, np.ones_like(v), 0.1)
+    assert np.allclose(out, 1.0, atol=1e-13)
+    # Q = 0 gives the mean of V over all keys
+    out, _ = O.joint_attention(np.zeros_like(q), k, v, 0.1)
+    assert np.allclose(out, v.mean(axis=1, keepdims=True), atol=1e-13)
+    # one key: O = V
+    out, _ = O.joint_attention(q[:, :1], k[:, :1], v[:, :1], 0.1)
+    assert np.allclose(out, v[:, :1], atol=1e-15)
+    # permuting keys together with values leaves O unchanged
+    perm = rng.permutation(N)
+    o1, l1 = O.joint_attention(q, k, v, 0.1)
+    o2, l2 = O.joint_attention(q, k[:, perm], v[:, perm], 0.1, rows=np.arange(N))
+    assert np.allclose(o1, o2, atol=1e-13) and np.allclose(l1, l2, atol=1e-13)
+    # one dominant logit selects its value row
+    kd = k.copy()
+    kd[0, 17, :, :] = q[0, 3, :, :] * 50.0
+    out, _ = O.joint_attention(q, kd, v, 1.0, rows=[3])
+    assert np.allclose(out[0, 0], v[0, 17], atol=1e-12)
+
+
+def test_attention_sampled_rows_equal_full_rows():
+    rng = np.random.default_rng(12)
+    q, k, v = (rng.standard_normal((1, 50, 2, 128)) for _ in range(3))
+    rows = [0, 7, 49]
+    full, lf = O.joint_attention(q, k, v, 0.09)
+    part, lp = O.joint_attention(q, k, v, 0.09, rows=rows)
+    assert np.allclose(full[:, rows], part, rtol=0, atol=1e-14)
+    assert np.allclose(lf[:, :, rows], lp, rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------- input recipe ----
+
+def test_inputs_are_seeded_and_shaped():
+    w = I.WORKLOADS["tiny"]
+    a = I.make_qkv(w, 0)
+    b = I.make_qkv(w, 0)
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    assert a[0].shape == (1, 288, 2, 128) and a[0].dtype == torch.bfloat16
+    rows = I.sampled_rows(I.WORKLOADS["i2i_2048"], 256)
+    assert len(rows) == 256 and len(set(rows.tolist())) == 256
+    for t in (0, 511, 512, 512 + 16383, 512 + 16384, 33279):
+        assert t in rows
+    m = I.outlier_rows(I.WORKLOADS["t2i_2048"])
+    assert m.sum() == round(0.01 * m.size)
