@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""Joint text+image attention forward benchmark (B200, sm_100a).
+
+One step = the whole hot path on one batch of synthetic input: the prologue
+(RMSNorm + 2-D RoPE of Q and K) followed by the joint attention forward, on
+the 2048^2 text-to-image workload with classifier-free guidance batched as
+B=2 (24 heads of 128, 512 text tokens + a 128x128 latent grid = 16896 joint
+tokens).  The metric is attention TFLOP/s with FLOPs = 4 * B * H * N^2 * d.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun every rank runs its own independent batch (weak scaling, no
+data-path collective); the step time is the max over ranks.  Rank 0 prints
+one JSON line.  ``--impl reference`` times the float64 CPU oracle instead,
+on a bounded sample of the same workload, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from diffusion_transformer_joint_dit_b200 import inputs as I  # noqa: E402
+
+METRIC = "joint-attn fwd TFLOP/s & % tensor peak, 2048² T2I (16896 tok, 24×128)"
+UNIT = "TFLOP/s"
+WORKLOAD = "t2i_2048"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_bf16_t2i_2048.json")
+KERNEL_SOURCES = ["attn_bf16.cu", "sm100_ptx.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU oracle baseline budget (rank 0, N=1)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(w: I.Workload, extra=None):
+    cfg = {
+        "workload": (f"{w.name}: B={w.B} H={w.H} d={w.d} N_txt={w.n_txt} N_img={w.n_img} "
+                     f"({w.img_h}x{w.img_w}) N_ref={w.n_ref} -> N={w.N} joint tokens"),
+        "B": w.B, "H": w.H, "N": w.N, "d": w.d, "path": w.path,
+        "step": "jattn_prologue (RMSNorm + 2-D RoPE of Q, K; bf16) + jattn_fwd_bf16",
+        "l2": f"inputs larger than L2: Q, K, V {3 * w.B * w.N * w.H * w.d * 2 / 1e6:.0f} MB read per step",
+        "parallelism": "independent batch per GPU (weak scaling, no collective)",
+    }
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "diffusion_transformer_joint_dit_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_sha256") != kernel_source_sha():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = local_rank
+        if vis:
+            parts = [p.strip() for p in vis.split(",") if p.strip()]
+            if local_rank < len(parts) and parts[local_rank].isdigit():
+                idx = int(parts[local_rank])
+        self.idx = idx
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle ----
+
+def oracle_unit(w: I.Workload, q, k, v, b: int, h: int, rows):
+    """Oracle prologue + attention for one (b, h) on sampled query rows."""
+    import oracle as O
+    qs = q[b:b + 1, :, h:h + 1, :].float().numpy()
+    ks = k[b:b + 1, :, h:h + 1, :].float().numpy()
+    vs = v[b:b + 1, :, h:h + 1, :].float().numpy()
+    # The prologue runs on the whole (b, h) slice (every key needs K'); the
+    # attention only on the sampled query rows.
+    qp, kp = O.prologue(qs, ks, n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w, ref_h=w.ref_h, ref_w=w.ref_w,
+                        ref_row_offset=w.ref_row_offset, theta=w.theta, eps=w.eps)
+    O.joint_attention(O.bf16_round(qp), O.bf16_round(kp), vs, w.softmax_scale, rows=rows)
+    return 4.0 * len(rows) * w.N * w.d
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [int(i.get("num_threads", 0)) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(w: I.Workload, q, k, v, seconds: float):
+    rows_per_unit = 256
+    rows = I.sampled_rows(w, rows_per_unit)
+    units = [(b, h) for b in range(w.B) for h in range(w.H)]
+    flops, done, t0 = 0.0, 0, time.perf_counter()
+    while done < len(units) and (time.perf_counter() - t0) < seconds:
+        b, h = units[done]
+        flops += oracle_unit(w, q, k, v, b, h, rows)
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"float64 oracle (prologue of one (b,h) slice + attention of {rows_per_unit} sampled "
+                       f"query rows vs all {w.N} keys) on {done} of {len(units)} (b,h) pairs, {dt:.1f} s"),
+            "seconds": dt}
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    w = I.WORKLOADS[args.workload]
+    q, k, v = I.make_qkv(w, seed=0)
+    rows = I.sampled_rows(w, 256)
+    units = [(b, h) for b in range(w.B) for h in range(w.H)]
+    for i in range(args.warmup):
+        b, h = units[i % len(units)]
+        oracle_unit(w, q, k, v, b, h, rows)
+    flops, t0 = 0.0, time.perf_counter()
+    for i in range(args.steps):
+        b, h = units[(args.warmup + i) % len(units)]
+        flops += oracle_unit(w, q, k, v, b, h, rows)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = (f"each step: float64 oracle prologue of one (b,h) slice of {w.name} + attention of 256 "
+              f"sampled query rows vs all {w.N} keys")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, {"sample": sample}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# -------------------------------------------------------------------- ours ----
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    from diffusion_transformer_joint_dit_b200 import binding as J
+
+    dist = world > 1
+    torch.cuda.set_device(local_rank)
+    if dist:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    w = I.WORKLOADS[args.workload]
+    if w.path != "bf16":
+        raise SystemExit("bench.py times the BF16 path")
+    q, k, v = I.make_qkv(w, seed=rank)
+    dev = torch.device("cuda", local_rank)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    qp, kp, o = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(qd)
+    params = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps)
+    stream = torch.cuda.current_stream(dev)
+    s_handle = stream.cuda_stream
+
+    def prologue():
+        J.jattn_prologue(qd, kd, None, qp, kp, None, None, None, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref,
+                         w.d, J.JATTN_PROLOGUE_BF16, params, s_handle)
+
+    def attention():
+        J.jattn_fwd_bf16(qp, kp, vd, o, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d, w.softmax_scale,
+                         s_handle)
+
+    for _ in range(max(args.warmup, 3)):
+        prologue()
+        attention()
+    torch.cuda.synchronize(dev)
+    if J.jattn_device_status(s_handle) != J.JATTN_OK:
+        raise RuntimeError("device error word set during warm-up")
+
+    # ---- device-timed region: inputs resident in HBM ----
+    K = args.steps
+    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    pro_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)  # let the sampler take its first reading
+    e0.record(stream)
+    for i in range(K):
+        pro_ev[i][0].record(stream)
+        prologue()
+        pro_ev[i][1].record(stream)
+        att_ev[i][0].record(stream)
+        attention()
+        att_ev[i][1].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if dist:
+        torch.distributed.barrier()
+    elapsed = e0.elapsed_time(e1)
+    att_ms = statistics.mean(a.elapsed_time(b) for a, b in att_ev)
+    pro_ms = statistics.mean(a.elapsed_time(b) for a, b in pro_ev)
+    if J.jattn_device_status(s_handle) != J.JATTN_OK:
+        raise RuntimeError("device error word set during timed steps")
+
+    # ---- end-to-end region: host buffers, copies inside the timed region ----
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    Ke = max(3, K // 5)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    f0.record(stream)
+    for _ in range(Ke):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        prologue()
+        attention()
+        oh.copy_(o, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_elapsed = f0.elapsed_time(f1)
+
+    times = torch.tensor([elapsed, e2e_elapsed, att_ms, pro_ms], dtype=torch.float64, device=dev)
+    if dist:
+        torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
+    elapsed, e2e_elapsed, att_ms, pro_ms = times.tolist()
+    if dist:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    ms_per_step = elapsed / K
+    value = world * w.flops / (ms_per_step * 1e-3) / 1e12
+    e2e_value = world * w.flops / (e2e_elapsed / Ke * 1e-3) / 1e12
+    peaks, peaks_src = load_peaks()
+    sustained = elapsed >= 1000.0
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    achieved = w.flops / (att_ms * 1e-3) / 1e12
+    traffic = profiled_traffic()
+    act_bytes = w.B * w.N * w.H * w.d * 2
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q, K, V; random-free kernels)",
+        "config": workload_config(w, {"attention_ms": att_ms, "prologue_ms": pro_ms,
+                                      "prologue_gbs": 4 * act_bytes / (pro_ms * 1e-3) / 1e9}),
+        "roofline": {
+            "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic,
+            "kernel": "attn_bf16_kernel", "flops_per_launch": w.flops,
+            "peak_source": f"{peaks_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}"
+                           f" ({'timed region >= 1 s' if sustained else 'timed region < 1 s'})",
+            "algorithmic_bytes_per_launch": 4 * act_bytes,
+        },
+        "prologue_roofline": {
+            "bound": "hbm", "achieved": 4 * act_bytes / (pro_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": 4 * act_bytes / (pro_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        },
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 3 * act_bytes,
+                "d2h_bytes_per_step": act_bytes, "steps": Ke},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k_: v_ for k_, v_ in cpu_baseline(w, q, k, v, args.cpu_seconds).items()
+                                if k_ != "seconds"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        raise SystemExit("--gpus N > 1 runs under torchrun (one process per GPU)")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

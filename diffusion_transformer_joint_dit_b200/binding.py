@@ -1,0 +1,157 @@
+"""ctypes binding of the jattn C-ABI (``include/jattn.h``).
+
+Argument marshalling only: every function forwards to the symbol of the same
+name in ``_lib/libjattn.so``, whose CUDA kernels do all of the work.  Tensor
+arguments may be torch tensors (their ``data_ptr()`` is passed), plain
+integer addresses or ``None`` (NULL).  ``stream`` may be a
+``torch.cuda.Stream``, an integer ``cudaStream_t`` handle, or ``None`` for
+torch's current stream on the current device.  A non-OK status raises
+:class:`JattnError`.  The library is loaded on first use; if it is missing or
+cannot be loaded the call raises: there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libjattn.so")
+
+JATTN_OK = 0
+JATTN_ERR_INVALID_ARG = 1
+JATTN_ERR_UNSUPPORTED = 2
+JATTN_ERR_MISALIGNED = 3
+JATTN_ERR_CUDA = 4
+JATTN_ERR_TIMEOUT = 5
+JATTN_PROLOGUE_BF16 = 0
+JATTN_PROLOGUE_FP8 = 1
+JATTN_FP8_BLOCK = 64
+
+EXPORTED = ("jattn_prologue", "jattn_fwd_bf16", "jattn_fwd_fp8", "jattn_status_string",
+            "jattn_device_status", "jattn_selftest_wait_timeout")
+
+
+class JattnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_name(status)} ({status})")
+
+
+class jattn_prologue_params(ctypes.Structure):
+    _fields_ = [
+        ("img_h", ctypes.c_int), ("img_w", ctypes.c_int),
+        ("ref_h", ctypes.c_int), ("ref_w", ctypes.c_int),
+        ("ref_row_offset", ctypes.c_int),
+        ("rope_theta", ctypes.c_float), ("eps", ctypes.c_float),
+        ("q_norm_w", ctypes.c_void_p), ("k_norm_w", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+def load_library():
+    """Load ``libjattn.so`` (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"jattn CUDA library not built: {LIB_PATH} is missing "
+                           "(run `python -c 'import __graft_entry__ as g; g.build()'`)")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.jattn_prologue.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                   ctypes.POINTER(jattn_prologue_params), _P]
+    lib.jattn_prologue.restype = _I
+    lib.jattn_fwd_bf16.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]
+    lib.jattn_fwd_bf16.restype = _I
+    lib.jattn_fwd_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]
+    lib.jattn_fwd_fp8.restype = _I
+    lib.jattn_status_string.argtypes = [_I]
+    lib.jattn_status_string.restype = ctypes.c_char_p
+    lib.jattn_device_status.argtypes = [_P]
+    lib.jattn_device_status.restype = _I
+    lib.jattn_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _P]
+    lib.jattn_selftest_wait_timeout.restype = _I
+    _lib = lib
+    return lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(fn: str, status: int) -> None:
+    if status != JATTN_OK:
+        raise JattnError(fn, status)
+
+
+def status_name(status: int) -> str:
+    return load_library().jattn_status_string(int(status)).decode()
+
+
+def jattn_status_string(status: int) -> str:
+    return status_name(status)
+
+
+def make_prologue_params(img_h: int, img_w: int, ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0,
+                         rope_theta: float = 10000.0, eps: float = 1e-6, q_norm_w=None, k_norm_w=None):
+    return jattn_prologue_params(img_h, img_w, ref_h, ref_w, ref_row_offset, rope_theta, eps,
+                                 _ptr(q_norm_w), _ptr(k_norm_w))
+
+
+def jattn_prologue(q, k, v, q_out, k_out, v_out, q_scale, k_scale, v_scale,
+                   B: int, H: int, N_txt: int, N_img: int, N_ref: int, d: int, mode: int,
+                   params: jattn_prologue_params, stream=None, *, check: bool = True) -> int:
+    st = load_library().jattn_prologue(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(q_out), _ptr(k_out), _ptr(v_out),
+        _ptr(q_scale), _ptr(k_scale), _ptr(v_scale),
+        B, H, N_txt, N_img, N_ref, d, mode,
+        ctypes.byref(params) if params is not None else None, _stream(stream))
+    if check:
+        _check("jattn_prologue", st)
+    return st
+
+
+def jattn_fwd_bf16(q, k, v, o, lse, B: int, H: int, N_txt: int, N_img: int, N_ref: int, d: int,
+                   softmax_scale: float, stream=None, *, check: bool = True) -> int:
+    st = load_library().jattn_fwd_bf16(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                       B, H, N_txt, N_img, N_ref, d, softmax_scale, _stream(stream))
+    if check:
+        _check("jattn_fwd_bf16", st)
+    return st
+
+
+def jattn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B: int, H: int, N_txt: int, N_img: int,
+                  N_ref: int, d: int, softmax_scale: float, stream=None, *, check: bool = True) -> int:
+    st = load_library().jattn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(q_scale), _ptr(k_scale),
+                                      _ptr(v_scale), _ptr(o), _ptr(lse), B, H, N_txt, N_img, N_ref, d,
+                                      softmax_scale, _stream(stream))
+    if check:
+        _check("jattn_fwd_fp8", st)
+    return st
+
+
+def jattn_device_status(stream=None) -> int:
+    return load_library().jattn_device_status(_stream(stream))
+
+
+def jattn_selftest_wait_timeout(timeout_ns: int, stream=None, *, check: bool = True) -> int:
+    st = load_library().jattn_selftest_wait_timeout(int(timeout_ns), _stream(stream))
+    if check:
+        _check("jattn_selftest_wait_timeout", st)
+    return st

@@ -1,0 +1,390 @@
+// Joint attention forward, BF16 operands, for sm_100a.
+//
+// O = softmax(scale * Q K^T) V over the whole joint [text | image | ref]
+// sequence of one (batch, head); the operation the NVIDIA tutorial on
+// FLUX 3 Image Klein ("Quantized and sparse attention" section) calls
+// VANILLA BF16 attention, the largest share of DiT GPU time at 2048^2.
+//
+// Design (one CTA = 256 query rows of one (b, h) = two 128-row Q tiles):
+//   warps 0-3  softmax for Q tile 0 (TMEM S0 / O0), then its epilogue
+//   warps 4-7  softmax for Q tile 1 (TMEM S1 / O1), then its epilogue
+//   warp 8     TMA producer: Q tiles once, then K_j, V_j into a ring of
+//              32 KB shared-memory slots (128-byte swizzle, two 64-channel
+//              boxes per 128-row tile)
+//   warp 9     TMEM allocator and the single thread issuing tcgen05.mma
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384)
+// O1 [384,512), all fp32 with TMEM lane = query row.  P_i (bf16, packed two
+// per column) overwrites columns [0,64) of S_i and feeds the P.V MMA
+// straight from TMEM.
+//
+// Per KV tile j the MMA thread issues, in order,
+//   PV0_j, QK0_{j+1}, PV1_j, QK1_{j+1}
+// so that while one softmax warpgroup works on its S tile the tensor core
+// runs the other tile's MMAs.  tcgen05.mma ops of one thread execute in
+// issue order, so QK_{j+1} writing S_i/P_i after PV_j read P_i is safe, and
+// the commit that signals S_i(j+1) also covers PV_i(j): the softmax may then
+// rescale O_i and overwrite P_i.
+//
+// Online softmax in the exp2 domain with a lazy maximum: the reference max
+// m of a row only moves when the new tile's max exceeds it by more than 8
+// (log2 units); P is then at most 2^8, harmless for bf16 P and fp32 O / l.
+// The O rescale (a TMEM read-modify-write) is thus rare after the first
+// tiles.  Tail keys (N not a multiple of 128) are masked to -inf; tail
+// query rows read zero-filled Q and are not stored.
+#include "jattn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace jattn {
+
+namespace bf16attn {
+
+constexpr int kBM = 128;           // query rows per Q tile (= TMEM lanes)
+constexpr int kTiles = 2;          // Q tiles per CTA
+constexpr int kBN = 128;           // keys per KV tile
+constexpr int kD = 128;            // head dim
+constexpr int kStages = 4;         // K/V ring slots
+constexpr int kTileBytes = kBM * kD * 2;       // 32 KB
+constexpr int kBoxBytes = kTileBytes / 2;      // 16 KB: 128 rows x 64 channels
+constexpr int kSoftmaxWarps = 4 * kTiles;
+constexpr int kLoadWarp = kSoftmaxWarps;       // 8
+constexpr int kMmaWarp = kSoftmaxWarps + 1;    // 9
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+
+struct Ctrl {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[kTiles];
+  uint64_t p_full[kTiles];
+  uint64_t o_full;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr int kSmemQ = 0;
+constexpr int kSmemRing = kTiles * kTileBytes;
+constexpr int kSmemCtrl = kSmemRing + kStages * kTileBytes;
+constexpr int kSmemBytes = kSmemCtrl + static_cast<int>(sizeof(Ctrl)) + 1024;  // + alignment slack
+
+struct Params {
+  __nv_bfloat16* o;
+  float* lse;
+  int H, N;
+  float scale_log2;
+  uint64_t timeout_ns;
+};
+
+// Wait that only gives up on time (used while draining at teardown).
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  int never = 0;
+  return mbar_wait(bar, parity, &never, timeout_ns);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params prm) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kSmemCtrl);
+  volatile int* abort_flag = &ctrl->abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int m0 = blockIdx.x * (kBM * kTiles);
+  const int N = prm.N;
+  const int n_kv = (N + kBN - 1) / kBN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctrl->kv_full[s], 1);
+      mbar_init(&ctrl->kv_empty[s], 1);
+    }
+    for (int t = 0; t < kTiles; ++t) {
+      mbar_init(&ctrl->s_full[t], 1);
+      mbar_init(&ctrl->p_full[t], 4 * 32);
+    }
+    mbar_init(&ctrl->o_full, 1);
+    mbar_init(&ctrl->mma_done, 1);
+    ctrl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&ctrl->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------ TMA producer ----
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      mbar_arrive_expect_tx(&ctrl->q_full, kTiles * kTileBytes);
+      for (int t = 0; t < kTiles; ++t) {
+        uint8_t* dst = smem + kSmemQ + t * kTileBytes;
+        tma_load_4d(dst, &tm_q, &ctrl->q_full, 0, h, m0 + t * kBM, b);
+        tma_load_4d(dst + kBoxBytes, &tm_q, &ctrl->q_full, 64, h, m0 + t * kBM, b);
+      }
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        for (int which = 0; which < 2; ++which, ++it) {
+          const int slot = it % kStages;
+          const uint32_t round = static_cast<uint32_t>(it / kStages);
+          if (!mbar_wait(&ctrl->kv_empty[slot], (round & 1u) ^ 1u, abort_flag, prm.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          const CUtensorMap* map = which == 0 ? &tm_k : &tm_v;
+          uint8_t* dst = smem + kSmemRing + slot * kTileBytes;
+          mbar_arrive_expect_tx(&ctrl->kv_full[slot], kTileBytes);
+          tma_load_4d(dst, map, &ctrl->kv_full[slot], 0, h, j * kBN, b);
+          tma_load_4d(dst + kBoxBytes, map, &ctrl->kv_full[slot], 64, h, j * kBN, b);
+        }
+      }
+      // Drain: every fill issued has landed before the CTA may exit.
+      drain_wait(&ctrl->q_full, 0, prm.timeout_ns);
+      for (int s = 0; s < kStages && s < it; ++s) {
+        const int last = s + ((it - 1 - s) / kStages) * kStages;  // last fill index of slot s
+        drain_wait(&ctrl->kv_full[s], static_cast<uint32_t>(last / kStages) & 1u, prm.timeout_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------- MMA issuer ----
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc(1, 1, false, kBM, kBN);  // bf16 x bf16, K-major both
+      constexpr uint32_t idesc_pv = make_idesc(1, 1, true, kBM, kD);    // P (TMEM) x V (MN-major)
+      const uint32_t q_base = smem_u32(smem + kSmemQ);
+      const uint32_t ring = smem_u32(smem + kSmemRing);
+
+      auto issue_qk = [&](int t, int slot) {
+        const uint32_t d = tmem + t * kBN;  // S_t
+        const uint32_t qa = q_base + t * kTileBytes;
+        const uint32_t kb = ring + slot * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          mma_f16_ss(d, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), idesc_qk,
+                     kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t d = tmem + 2 * kBN + t * kD;  // O_t
+        const uint32_t p = tmem + t * kBN;           // P_t (packed bf16 in S_t columns)
+        const uint32_t vb = ring + slot * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          mma_f16_ts(d, p + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, kBoxBytes, 1024), idesc_pv,
+                     (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = mbar_wait(&ctrl->q_full, 0, abort_flag, prm.timeout_ns);
+      int it = 0;
+      if (ok) ok = mbar_wait(&ctrl->kv_full[0], 0, abort_flag, prm.timeout_ns);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 0);
+        mma_commit(&ctrl->s_full[0]);
+        issue_qk(1, 0);
+        mma_commit(&ctrl->s_full[1]);
+        mma_commit(&ctrl->kv_empty[0]);
+        it = 1;
+      }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int slot_v = it % kStages;
+        ok = mbar_wait(&ctrl->kv_full[slot_v], static_cast<uint32_t>(it / kStages) & 1u, abort_flag,
+                       prm.timeout_ns);
+        ++it;
+        if (!ok) break;
+        const bool has_next = j + 1 < n_kv;
+        const int slot_k = it % kStages;
+        // Q tile 0
+        ok = mbar_wait(&ctrl->p_full[0], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, slot_v, j > 0);
+        if (has_next) {
+          ok = mbar_wait(&ctrl->kv_full[slot_k], static_cast<uint32_t>(it / kStages) & 1u, abort_flag,
+                         prm.timeout_ns);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(0, slot_k);
+          mma_commit(&ctrl->s_full[0]);
+        }
+        // Q tile 1
+        ok = mbar_wait(&ctrl->p_full[1], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(1, slot_v, j > 0);
+        mma_commit(&ctrl->kv_empty[slot_v]);
+        if (has_next) {
+          issue_qk(1, slot_k);
+          mma_commit(&ctrl->s_full[1]);
+          mma_commit(&ctrl->kv_empty[slot_k]);
+          ++it;
+        }
+      }
+      if (ok) mma_commit(&ctrl->o_full);
+      // Drain: all issued MMAs complete before TMEM is released.
+      mma_commit(&ctrl->mma_done);
+      drain_wait(&ctrl->mma_done, 0, prm.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------- softmax + epilogue (x2) ----
+    const int t = warp >> 2;                 // Q tile of this warpgroup
+    const int wq = warp & 3;                 // TMEM lane quarter
+    const int r = wq * 32 + lane;            // row within the tile
+    const uint32_t lane_sel = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t s_addr = tmem + lane_sel + t * kBN;
+    const uint32_t o_addr = tmem + lane_sel + 2 * kBN + t * kD;
+    const float sl2 = prm.scale_log2;
+
+    float m = -INFINITY;  // reference row max (log2 units of scaled logits)
+    float l = 0.f;        // row sum of exp2(x - m)
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      // Warp-uniform outcome: the tcgen05.ld/st below are warp-collective.
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&ctrl->s_full[t], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sv[c]);
+      tmem_ld_wait();
+
+      const int nvalid = N - j * kBN;  // >= 1
+      if (nvalid < kBN) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i >= nvalid) sv[c][i] = __float_as_uint(-INFINITY);
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        mx0 = fmaxf(mx0, __uint_as_float(sv[0][i]));
+        mx1 = fmaxf(mx1, __uint_as_float(sv[1][i]));
+        mx2 = fmaxf(mx2, __uint_as_float(sv[2][i]));
+        mx3 = fmaxf(mx3, __uint_as_float(sv[3][i]));
+      }
+      const float mnew = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+      const bool need = mnew > m + kRescaleThreshold;
+      float corr = 1.f;
+      if (need) {
+        corr = ex2_approx(m - mnew);  // 0 on the first tile
+        l *= corr;
+        m = mnew;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(o_addr + c * 32, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+          tmem_st32(o_addr + c * 32, ov);
+        }
+      }
+      // P = exp2(x - m), packed two bf16 per 32-bit word in place: keys
+      // [0,64) land in sv[0], keys [64,128) in sv[2] (each packed word is
+      // written at or before the index it was read from).
+      const float neg_m = -m;
+      float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c][i]), sl2, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c][i + 1]), sl2, neg_m));
+          l0 += p0;
+          l1 += p1;
+          sv[c & 2][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
+        }
+      }
+      l += l0 + l1;
+      tmem_st32(s_addr, sv[0]);
+      tmem_st32(s_addr + 32, sv[2]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ctrl->p_full[t]);
+    }
+
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->o_full, 0, abort_flag, prm.timeout_ns))) {
+      tc_fence_after();
+      const int row = m0 + t * kBM + r;
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* orow = prm.o + ((static_cast<size_t>(b) * N + row) * prm.H + h) * kD;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(o_addr + c * 32, ov);
+        tmem_ld_wait();
+        if (row < N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(ov[8 * q4 + 0]) * inv_l, __uint_as_float(ov[8 * q4 + 1]) * inv_l);
+            u.y = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2]) * inv_l, __uint_as_float(ov[8 * q4 + 3]) * inv_l);
+            u.z = pack_bf16x2(__uint_as_float(ov[8 * q4 + 4]) * inv_l, __uint_as_float(ov[8 * q4 + 5]) * inv_l);
+            u.w = pack_bf16x2(__uint_as_float(ov[8 * q4 + 6]) * inv_l, __uint_as_float(ov[8 * q4 + 7]) * inv_l);
+            dst[q4] = u;
+          }
+        }
+      }
+      if (prm.lse != nullptr && row < N) {
+        prm.lse[(static_cast<size_t>(b) * prm.H + h) * N + row] = (m + __log2f(l)) * 0.69314718055994530942f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace bf16attn
+
+
+cudaError_t launch_attn_bf16(const AttnProblem& p, cudaStream_t s) {
+  using namespace bf16attn;
+  CUtensorMap tq, tk, tv;
+  cudaError_t e;
+  if ((e = make_act_map(&tq, p.q, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
+  if ((e = make_act_map(&tk, p.k, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
+  if ((e = make_act_map(&tv, p.v, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
+  if ((e = set_smem_attr(reinterpret_cast<const void*>(attn_bf16_kernel), kSmemBytes)) != cudaSuccess) return e;
+  Params prm;
+  prm.o = static_cast<__nv_bfloat16*>(p.o);
+  prm.lse = p.lse;
+  prm.H = p.H;
+  prm.N = p.N;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(p.softmax_scale) * 1.4426950408889634074);
+  prm.timeout_ns = p.timeout_ns;
+  dim3 grid((p.N + kBM * kTiles - 1) / (kBM * kTiles), p.H, p.B);
+  attn_bf16_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, prm);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace jattn

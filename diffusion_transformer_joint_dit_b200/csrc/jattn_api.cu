@@ -1,0 +1,238 @@
+// C-ABI of the jattn library (declared in include/jattn.h): argument
+// checks, tensor-map encoding and kernel launches.  Built as one
+// translation unit with the kernels so that device globals need no
+// relocatable device code.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "jattn.h"
+#include "jattn_internal.h"
+#include "sm100_ptx.cuh"
+
+#include "attn_bf16.cu"
+#include "attn_fp8.cu"
+#include "prologue.cu"
+
+namespace jattn {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+  });
+  return fn;
+}
+
+// Wait-timeout self test: one thread waits on a barrier nothing completes.
+__global__ void wait_selftest_kernel(uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, timeout_ns);
+  __syncthreads();
+}
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+
+int map_err(cudaError_t e) { return e == cudaSuccess ? JATTN_OK : JATTN_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int N_txt, int N_img, int N_ref, int d) {
+  if (B < 1 || H < 1 || N_txt < 0 || N_img < 0 || N_ref < 0) return JATTN_ERR_INVALID_ARG;
+  if (B > 65535 || H > 65535) return JATTN_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(N_txt) + N_img + N_ref;
+  if (N < 1 || N > (1ll << 30)) return JATTN_ERR_INVALID_ARG;
+  if (d != kHeadDim) return JATTN_ERR_UNSUPPORTED;
+  // Element offsets are formed in 64 bits; keep B*N*H*d within int64 and
+  // each tensor below 2^40 bytes (TMA global stride limit).
+  if (static_cast<long long>(B) * N * H * d * 2 >= (1ll << 40)) return JATTN_ERR_INVALID_ARG;
+  return JATTN_OK;
+}
+
+}  // namespace
+
+cudaError_t make_act_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int elem_bytes) {
+  EncodeTiledFn fn = encoder();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t row = static_cast<cuuint64_t>(kHeadDim) * elem_bytes;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {row, row * H, row * H * N};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = fn(map, dt, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t set_smem_attr(const void* func, int bytes) {
+  constexpr int kMaxDev = 64;
+  constexpr int kMaxFuncs = 8;
+  static std::mutex mu;
+  static const void* done_func[kMaxDev][kMaxFuncs] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < kMaxDev) {
+    for (int i = 0; i < kMaxFuncs; ++i)
+      if (done_func[dev][i] == func) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDev) {
+    for (int i = 0; i < kMaxFuncs; ++i)
+      if (done_func[dev][i] == nullptr) {
+        done_func[dev][i] = func;
+        break;
+      }
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(timeout_ns);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace jattn
+
+using namespace jattn;
+
+extern "C" {
+
+const char* jattn_status_string(int status) {
+  switch (status) {
+    case JATTN_OK: return "JATTN_OK";
+    case JATTN_ERR_INVALID_ARG: return "JATTN_ERR_INVALID_ARG";
+    case JATTN_ERR_UNSUPPORTED: return "JATTN_ERR_UNSUPPORTED";
+    case JATTN_ERR_MISALIGNED: return "JATTN_ERR_MISALIGNED";
+    case JATTN_ERR_CUDA: return "JATTN_ERR_CUDA";
+    case JATTN_ERR_TIMEOUT: return "JATTN_ERR_TIMEOUT";
+    default: return "JATTN_ERR_UNKNOWN";
+  }
+}
+
+int jattn_prologue(const void* q, const void* k, const void* v, void* q_out, void* k_out, void* v_out,
+                   float* q_scale, float* k_scale, float* v_scale, int B, int H, int N_txt, int N_img, int N_ref,
+                   int d, int mode, const jattn_prologue_params* p, void* cuda_stream) {
+  int st = check_common(B, H, N_txt, N_img, N_ref, d);
+  if (st != JATTN_OK) return st;
+  if (p == nullptr || (mode != JATTN_PROLOGUE_BF16 && mode != JATTN_PROLOGUE_FP8)) return JATTN_ERR_INVALID_ARG;
+  if (p->img_h < 0 || p->img_w < 0 || p->ref_h < 0 || p->ref_w < 0 || p->ref_row_offset < 0)
+    return JATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(p->img_h) * p->img_w != N_img || static_cast<long long>(p->ref_h) * p->ref_w != N_ref)
+    return JATTN_ERR_INVALID_ARG;
+  if (!(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta) || !(p->eps >= 0.f) || !std::isfinite(p->eps))
+    return JATTN_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || q_out == nullptr || k_out == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return JATTN_ERR_MISALIGNED;
+  if (!aligned16(p->q_norm_w) || !aligned16(p->k_norm_w)) return JATTN_ERR_MISALIGNED;
+  if (mode == JATTN_PROLOGUE_FP8) {
+    if (v == nullptr || v_out == nullptr || q_scale == nullptr || k_scale == nullptr || v_scale == nullptr)
+      return JATTN_ERR_INVALID_ARG;
+    if (!aligned16(v) || !aligned16(v_out)) return JATTN_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
+         reinterpret_cast<uintptr_t>(v_scale)) & 3u)
+      return JATTN_ERR_MISALIGNED;
+  }
+  PrologueArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v;
+  a.q_out = q_out; a.k_out = k_out; a.v_out = v_out;
+  a.q_scale = q_scale; a.k_scale = k_scale; a.v_scale = v_scale;
+  a.q_w = p->q_norm_w; a.k_w = p->k_norm_w;
+  a.B = B; a.H = H; a.N = N_txt + N_img + N_ref;
+  a.n_txt = N_txt; a.n_img = N_img;
+  a.img_w = p->img_w > 0 ? p->img_w : 1;
+  a.ref_w = p->ref_w > 0 ? p->ref_w : 1;
+  a.ref_row_offset = p->ref_row_offset;
+  a.eps = p->eps;
+  for (int i = 0; i < 32; ++i) a.omega[i] = std::pow(static_cast<double>(p->rope_theta), -2.0 * i / 64.0);
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  return map_err(mode == JATTN_PROLOGUE_BF16 ? launch_prologue_bf16(a, s) : launch_prologue_fp8(a, s));
+}
+
+int jattn_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N_txt,
+                   int N_img, int N_ref, int d, float softmax_scale, void* cuda_stream) {
+  int st = check_common(B, H, N_txt, N_img, N_ref, d);
+  if (st != JATTN_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return JATTN_ERR_MISALIGNED;
+  AttnProblem pr;
+  std::memset(&pr, 0, sizeof(pr));
+  pr.q = q; pr.k = k; pr.v = v; pr.o = o; pr.lse = lse;
+  pr.B = B; pr.H = H; pr.N = N_txt + N_img + N_ref;
+  pr.softmax_scale = softmax_scale;
+  pr.timeout_ns = kDefaultTimeoutNs;
+  return map_err(launch_attn_bf16(pr, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+int jattn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+                  const float* v_scale, void* o, float* lse, int B, int H, int N_txt, int N_img, int N_ref, int d,
+                  float softmax_scale, void* cuda_stream) {
+  int st = check_common(B, H, N_txt, N_img, N_ref, d);
+  if (st != JATTN_OK) return st;
+  if (q8 == nullptr || k8 == nullptr || v8 == nullptr || o == nullptr || q_scale == nullptr ||
+      k_scale == nullptr || v_scale == nullptr)
+    return JATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) ||
+      ((reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(q_scale) |
+        reinterpret_cast<uintptr_t>(k_scale) | reinterpret_cast<uintptr_t>(v_scale)) & 3u))
+    return JATTN_ERR_MISALIGNED;
+  AttnProblem pr;
+  std::memset(&pr, 0, sizeof(pr));
+  pr.q = q8; pr.k = k8; pr.v = v8;
+  pr.q_scale = q_scale; pr.k_scale = k_scale; pr.v_scale = v_scale;
+  pr.o = o; pr.lse = lse;
+  pr.B = B; pr.H = H; pr.N = N_txt + N_img + N_ref;
+  pr.softmax_scale = softmax_scale;
+  pr.timeout_ns = kDefaultTimeoutNs;
+  cudaError_t e = launch_attn_fp8(pr, static_cast<cudaStream_t>(cuda_stream));
+  if (e == cudaErrorNotSupported) return JATTN_ERR_UNSUPPORTED;
+  return map_err(e);
+}
+
+int jattn_device_status(void* cuda_stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return JATTN_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return JATTN_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return JATTN_ERR_CUDA;
+    return JATTN_ERR_TIMEOUT;
+  }
+  return JATTN_OK;
+}
+
+int jattn_selftest_wait_timeout(long long timeout_ns, void* cuda_stream) {
+  if (timeout_ns < 1 || timeout_ns > 1000000000ll) return JATTN_ERR_INVALID_ARG;
+  return map_err(launch_wait_selftest(static_cast<uint64_t>(timeout_ns), static_cast<cudaStream_t>(cuda_stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal launch interface between the C-ABI layer (jattn_api.cu) and the
+// kernels.  Not installed; not part of the public C-ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace jattn {
+
+constexpr int kHeadDim = 128;
+constexpr int kQuantBlock = 64;
+
+// Arguments of the prologue kernels, passed by value (__grid_constant__).
+struct PrologueArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* q_out;
+  void* k_out;
+  void* v_out;
+  float* q_scale;
+  float* k_scale;
+  float* v_scale;
+  const float* q_w;  // nullable: weight 1.0
+  const float* k_w;
+  int B, H, N;
+  int n_txt, n_img, img_w, ref_w, ref_row_offset;
+  float eps;
+  // RoPE frequencies of the 32 channel pairs of one axis half,
+  // omega_i = theta^(-2i/64), in double so that angles are exact enough.
+  double omega[32];
+};
+
+cudaError_t launch_prologue_bf16(const PrologueArgs& a, cudaStream_t s);
+cudaError_t launch_prologue_fp8(const PrologueArgs& a, cudaStream_t s);
+
+struct AttnProblem {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* q_scale;  // fp8 only
+  const float* k_scale;
+  const float* v_scale;
+  void* o;
+  float* lse;  // nullable
+  int B, H, N;
+  float softmax_scale;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_attn_bf16(const AttnProblem& p, cudaStream_t s);
+cudaError_t launch_attn_fp8(const AttnProblem& p, cudaStream_t s);
+cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t s);
+
+// 4-D tensor map over a token-major [B, N, H, d=128] tensor with
+// `elem_bytes`-byte elements (2 = bf16, 1 = e4m3): dims (d, H, N, B), box
+// (128 bytes of channels, 1 head, 128 tokens, 1 batch), 128-byte swizzle,
+// zero fill out of bounds.  Encoded through cuTensorMapEncodeTiled, looked
+// up via the runtime's driver entry point (no link-time libcuda dependency).
+cudaError_t make_act_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int elem_bytes);
+
+// Raise a kernel's dynamic shared-memory limit on the current device (once
+// per device and kernel).
+cudaError_t set_smem_attr(const void* func, int bytes);
+
+}  // namespace jattn

@@ -1,0 +1,325 @@
+// Prologue of the joint attention: per-head RMSNorm of Q and K, 2-D RoPE on
+// the tokens' (row, col) latent-grid positions, and (FP8 mode) E4M3 block
+// quantisation of Q', K' and V with one scale per (batch, head, 64 tokens).
+//
+// Source of the operation: the QKV projection epilogue that applies
+// query/key normalisation and rotary position embedding ("GEMM kernel
+// optimization" section of the NVIDIA tutorial on accelerating FLUX 3 Image
+// Klein with TensorRT LLM VisualGen) and FP8 Q/K/V attention inputs
+// ("Quantized and sparse attention" section of the same tutorial).
+//
+// Memory-bound.  Rows of 128 bf16 channels (256 B) are read with 128-bit
+// loads, one row per half-warp: lane l16 = lane % 16 owns channels
+// [8*l16, 8*l16 + 8).  Lanes 0-7 of a half hold the row-position half of
+// the head (channels 0-63), lanes 8-15 the column-position half, so each
+// lane rotates 4 self-contained adjacent pairs.  Row sums of squares are
+// reduced with 4 xor-shuffles inside the half-warp.
+#include <cuda_fp8.h>
+
+#include "jattn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace jattn {
+
+namespace {
+
+// (row, col) RoPE position of joint-sequence token t.
+__device__ __forceinline__ void token_pos(const PrologueArgs& a, int t, int& row, int& col) {
+  if (t < a.n_txt) {
+    row = 0;
+    col = 0;
+  } else if (t < a.n_txt + a.n_img) {
+    const int u = t - a.n_txt;
+    row = u / a.img_w;
+    col = u - row * a.img_w;
+  } else {
+    const int u = t - a.n_txt - a.n_img;
+    const int r = u / a.ref_w;
+    row = a.ref_row_offset + r;
+    col = u - r * a.ref_w;
+  }
+}
+
+// cos / sin of pos * omega for the lane's 4 channel pairs.  The angle is
+// formed and reduced to [-pi, pi] in double, then evaluated in float.
+__device__ __forceinline__ void lane_rotations(const PrologueArgs& a, int pos, int pair0, float (&c)[4],
+                                               float (&s)[4]) {
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const double phi = static_cast<double>(pos) * a.omega[pair0 + m];
+    const double r = phi - rint(phi * kInvTwoPi) * kTwoPi;
+    sincosf(static_cast<float>(r), &s[m], &c[m]);
+  }
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
+  uint4 u;
+  u.x = pack_bf16x2(y[0], y[1]);
+  u.y = pack_bf16x2(y[2], y[3]);
+  u.z = pack_bf16x2(y[4], y[5]);
+  u.w = pack_bf16x2(y[6], y[7]);
+  return u;
+}
+
+// RMSNorm over the half-warp's row, weight, then rotate the lane's 4 pairs.
+// Returns the bf16-rounded result packed.  `valid` rows contribute zeros to
+// nothing: every lane of a half-warp shares the same validity.
+__device__ __forceinline__ uint4 norm_rope_row(const uint4& raw, const float (&w)[8], const float (&c)[4],
+                                               const float (&s)[4], float eps) {
+  float x[8];
+  unpack8(raw, x);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+  const float r = rsqrtf(ss * (1.0f / kHeadDim) + eps);
+  float y[8];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const float a0 = x[2 * m] * r * w[2 * m];
+    const float a1 = x[2 * m + 1] * r * w[2 * m + 1];
+    y[2 * m] = fmaf(a0, c[m], -a1 * s[m]);
+    y[2 * m + 1] = fmaf(a0, s[m], a1 * c[m]);
+  }
+  return pack8(y);
+}
+
+__device__ __forceinline__ void load_weights(const float* w, int l16, float (&out)[8]) {
+  if (w == nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = 1.f;
+  } else {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(w + 8 * l16));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(w + 8 * l16 + 4));
+    out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+    out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+  }
+}
+
+// ------------------------------------------------------------ BF16 mode ----
+// One warp per (b, token); heads in batches of kRows per half-warp, Q and K
+// together, so the lane's 4 rotations are computed once per token.
+constexpr int kBf16Warps = 8;
+constexpr int kRows = 4;
+
+__global__ void __launch_bounds__(kBf16Warps * 32) prologue_bf16_kernel(const __grid_constant__ PrologueArgs a) {
+  const int lane = threadIdx.x & 31;
+  const long long token = static_cast<long long>(blockIdx.x) * kBf16Warps + (threadIdx.x >> 5);
+  if (token >= static_cast<long long>(a.B) * a.N) return;
+  const int t = static_cast<int>(token % a.N);
+  const int half = lane >> 4;
+  const int l16 = lane & 15;
+  const int axis = l16 >> 3;
+  const int pair0 = (l16 & 7) * 4;
+
+  int row, col;
+  token_pos(a, t, row, col);
+  float c[4], s[4];
+  lane_rotations(a, axis == 0 ? row : col, pair0, c, s);
+  float wq[8], wk[8];
+  load_weights(a.q_w, l16, wq);
+  load_weights(a.k_w, l16, wk);
+
+  const size_t row_base = static_cast<size_t>(token) * a.H;  // row index of head 0
+  const uint4* qin = reinterpret_cast<const uint4*>(a.q);
+  const uint4* kin = reinterpret_cast<const uint4*>(a.k);
+  uint4* qout = reinterpret_cast<uint4*>(a.q_out);
+  uint4* kout = reinterpret_cast<uint4*>(a.k_out);
+
+  for (int h0 = 0; h0 < a.H; h0 += 2 * kRows) {
+    uint4 rq[kRows], rk[kRows];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      const int h = h0 + 2 * r + half;
+      const size_t idx = (row_base + h) * 16 + l16;
+      if (h < a.H) {
+        rq[r] = __ldcs(qin + idx);
+        rk[r] = __ldcs(kin + idx);
+      } else {
+        rq[r] = make_uint4(0, 0, 0, 0);
+        rk[r] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      const int h = h0 + 2 * r + half;
+      const uint4 yq = norm_rope_row(rq[r], wq, c, s, a.eps);
+      const uint4 yk = norm_rope_row(rk[r], wk, c, s, a.eps);
+      if (h < a.H) {
+        const size_t idx = (row_base + h) * 16 + l16;
+        qout[idx] = yq;
+        kout[idx] = yk;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------- FP8 mode ----
+// One CTA per (64-token block, group of 4 heads, batch); 16 warps, each
+// owning 4 tokens; a half-warp owns one head of a token.  Processed rows
+// stay in registers (bf16-rounded) while the block absmax is reduced in
+// shared memory, then are quantised and stored as E4M3.
+constexpr int kFp8Warps = 16;
+constexpr int kFp8TokPerWarp = kQuantBlock / kFp8Warps;  // 4
+constexpr int kFp8Heads = 4;
+constexpr int kFp8Pairs = kFp8Heads / 2;                 // head pairs per token
+
+__device__ __forceinline__ float absmax8(const uint4& u) {
+  // |bf16| as float: clear the sign bit of each half and compare as floats.
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = fmaxf(m, __uint_as_float((w[i] << 16) & 0x7FFFFFFFu));
+    m = fmaxf(m, __uint_as_float(w[i] & 0x7FFF0000u));
+  }
+  return m;
+}
+
+__device__ __forceinline__ uint2 quant8(const uint4& u, float inv) {
+  float x[8];
+  unpack8(u, x);
+  uint32_t out[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float2 f;
+      f.x = __fmul_rn(x[4 * i + 2 * j], inv);
+      f.y = __fmul_rn(x[4 * i + 2 * j + 1], inv);
+      const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+      word |= static_cast<uint32_t>(p) << (16 * j);
+    }
+    out[i] = word;
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+__global__ void __launch_bounds__(kFp8Warps * 32) prologue_fp8_kernel(const __grid_constant__ PrologueArgs a) {
+  __shared__ unsigned int s_amax[3][kFp8Heads];
+  __shared__ float s_inv[3][kFp8Heads];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4;
+  const int l16 = lane & 15;
+  const int axis = l16 >> 3;
+  const int pair0 = (l16 & 7) * 4;
+  const int blk = blockIdx.x;
+  const int hg = blockIdx.y * kFp8Heads;
+  const int b = blockIdx.z;
+  const int nblk = (a.N + kQuantBlock - 1) / kQuantBlock;
+
+  if (threadIdx.x < 3 * kFp8Heads) s_amax[threadIdx.x / kFp8Heads][threadIdx.x % kFp8Heads] = 0u;
+
+  float c[kFp8TokPerWarp][4], s[kFp8TokPerWarp][4];
+#pragma unroll
+  for (int k = 0; k < kFp8TokPerWarp; ++k) {
+    const int t = blk * kQuantBlock + warp * kFp8TokPerWarp + k;
+    int row = 0, col = 0;
+    if (t < a.N) token_pos(a, t, row, col);
+    lane_rotations(a, axis == 0 ? row : col, pair0, c[k], s[k]);
+  }
+  __syncthreads();
+
+  const void* ins[3] = {a.q, a.k, a.v};
+  void* outs[3] = {a.q_out, a.k_out, a.v_out};
+  float* scales[3] = {a.q_scale, a.k_scale, a.v_scale};
+  const float* wts[2] = {a.q_w, a.k_w};
+
+#pragma unroll 1
+  for (int ti = 0; ti < 3; ++ti) {
+    const uint4* in = reinterpret_cast<const uint4*>(ins[ti]);
+    uint4 rows[kFp8TokPerWarp][kFp8Pairs];
+#pragma unroll
+    for (int k = 0; k < kFp8TokPerWarp; ++k) {
+      const int t = blk * kQuantBlock + warp * kFp8TokPerWarp + k;
+#pragma unroll
+      for (int j = 0; j < kFp8Pairs; ++j) {
+        const int h = hg + 2 * j + half;
+        if (t < a.N && h < a.H) {
+          const size_t idx = ((static_cast<size_t>(b) * a.N + t) * a.H + h) * 16 + l16;
+          rows[k][j] = __ldcs(in + idx);
+        } else {
+          rows[k][j] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+    if (ti < 2) {
+      float w[8];
+      load_weights(wts[ti], l16, w);
+#pragma unroll
+      for (int k = 0; k < kFp8TokPerWarp; ++k)
+#pragma unroll
+        for (int j = 0; j < kFp8Pairs; ++j) rows[k][j] = norm_rope_row(rows[k][j], w, c[k], s[k], a.eps);
+    }
+    // Block absmax per head: lanes of a half-warp, 4 tokens, then the CTA.
+#pragma unroll
+    for (int j = 0; j < kFp8Pairs; ++j) {
+      float m = 0.f;
+#pragma unroll
+      for (int k = 0; k < kFp8TokPerWarp; ++k) m = fmaxf(m, absmax8(rows[k][j]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      if (l16 == 0) atomicMax(&s_amax[ti][2 * j + half], __float_as_uint(m));
+    }
+    __syncthreads();
+    if (threadIdx.x < kFp8Heads) {
+      const int h = hg + threadIdx.x;
+      const float amax = __uint_as_float(s_amax[ti][threadIdx.x]);
+      const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+      s_inv[ti][threadIdx.x] = inv;
+      if (h < a.H) {
+        scales[ti][(static_cast<size_t>(b) * a.H + h) * nblk + blk] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      }
+    }
+    __syncthreads();
+    uint2* out = reinterpret_cast<uint2*>(outs[ti]);
+#pragma unroll
+    for (int k = 0; k < kFp8TokPerWarp; ++k) {
+      const int t = blk * kQuantBlock + warp * kFp8TokPerWarp + k;
+#pragma unroll
+      for (int j = 0; j < kFp8Pairs; ++j) {
+        const int h = hg + 2 * j + half;
+        if (t < a.N && h < a.H) {
+          const size_t idx = ((static_cast<size_t>(b) * a.N + t) * a.H + h) * 16 + l16;
+          __stcs(out + idx, quant8(rows[k][j], s_inv[ti][2 * j + half]));
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prologue_bf16(const PrologueArgs& a, cudaStream_t s) {
+  const long long tokens = static_cast<long long>(a.B) * a.N;
+  const unsigned grid = static_cast<unsigned>((tokens + kBf16Warps - 1) / kBf16Warps);
+  prologue_bf16_kernel<<<grid, kBf16Warps * 32, 0, s>>>(a);
+  return cudaPeekAtLastError();
+}
+
+cudaError_t launch_prologue_fp8(const PrologueArgs& a, cudaStream_t s) {
+  dim3 grid((a.N + kQuantBlock - 1) / kQuantBlock, (a.H + kFp8Heads - 1) / kFp8Heads, a.B);
+  prologue_fp8_kernel<<<grid, kFp8Warps * 32, 0, s>>>(a);
+  return cudaPeekAtLastError();
+}
+
+}  // namespace jattn

@@ -1,0 +1,189 @@
+/*
+ * jattn — joint text + image (+ reference image) multi-head self-attention
+ * forward of one DiT block, for NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute.  The NVIDIA tutorial on accelerating FLUX 3 Image
+ * Klein with TensorRT LLM VisualGen ("FLUX 3 inference with TensorRT LLM
+ * VisualGen" section) describes a DiT that processes the text, noisy-target
+ * and optional reference-image token streams separately and lets them meet
+ * only in one joint attention.  Its "GEMM kernel optimization" section fuses
+ * query/key normalisation and rotary position embedding into the QKV
+ * projection epilogue; its "Quantized and sparse attention" section runs the
+ * attention itself either in BF16 or with FP8 Q/K and FP8 V.  The three
+ * calls below are those steps:
+ *
+ *   jattn_prologue   per-head RMSNorm of Q and K, 2-D RoPE on the tokens'
+ *                    (row, col) latent-grid positions, optionally followed
+ *                    by E4M3 block quantisation of Q', K' and V;
+ *   jattn_fwd_bf16   O = softmax(scale * Q' K'^T) V over the whole joint
+ *                    sequence (no mask), bf16 in, fp32 accumulate, bf16 out;
+ *   jattn_fwd_fp8    the same from E4M3 codes with per-64-token block scales.
+ *
+ * Layout.  Every activation tensor is token-major [B, N, H, d], the layout a
+ * QKV projection writes: element (b, t, h, c) sits at
+ * ((b * N + t) * H + h) * d + c.  The joint sequence is the concatenation
+ * [text (N_txt) | noisy target image (N_img) | reference image (N_ref)],
+ * N = N_txt + N_img + N_ref; the caller lays the streams out contiguously.
+ * Image tokens are the latent grid flattened row-major.
+ *
+ * Ownership and execution.  The caller owns all memory (device pointers
+ * unless stated otherwise).  The library never allocates, frees or
+ * synchronises inside these calls: each enqueues its kernel(s) on
+ * `cuda_stream` (a cudaStream_t; NULL = legacy default stream) and returns.
+ * Results are valid once the stream has run the work.
+ *
+ * Errors.  Arguments are checked before any launch; a rejected call launches
+ * nothing and returns a jattn_status below.  After a launch the return is the
+ * launch status (cudaPeekAtLastError) mapped to JATTN_ERR_CUDA.  Every wait
+ * inside the attention kernels is bounded; a wait that runs out sets a device
+ * error word and the kernel returns early, leaving its outputs undefined;
+ * jattn_device_status() reports and clears it.
+ */
+#ifndef JATTN_H_
+#define JATTN_H_
+
+#if defined(__GNUC__)
+#define JATTN_API __attribute__((visibility("default")))
+#else
+#define JATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  JATTN_OK = 0,
+  JATTN_ERR_INVALID_ARG = 1,  /* a size, pointer or enum out of range        */
+  JATTN_ERR_UNSUPPORTED = 2,  /* valid, but not built (e.g. head_dim != 128)  */
+  JATTN_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned             */
+  JATTN_ERR_CUDA = 4,         /* the CUDA runtime reported an error           */
+  JATTN_ERR_TIMEOUT = 5       /* a bounded in-kernel wait ran out             */
+} jattn_status;
+
+/* Prologue modes. */
+#define JATTN_PROLOGUE_BF16 0  /* Q', K' written as bf16; V untouched               */
+#define JATTN_PROLOGUE_FP8 1   /* Q', K', V written as E4M3 codes + block scales     */
+
+/* Token block covered by one FP8 scale (tokens of one (batch, head)). */
+#define JATTN_FP8_BLOCK 64
+
+/*
+ * Position and normalisation parameters of the prologue.
+ *
+ * RoPE positions (2-D, the reading of the workloads' "split 64/64 over
+ * (row, col)"): text token t < N_txt sits at (0, 0); image token
+ * t' = t - N_txt at (t' / img_w, t' % img_w); reference token
+ * t'' = t - N_txt - N_img at (ref_row_offset + t'' / ref_w, t'' % ref_w).
+ * Channels [0, d/2) rotate with the row position, [d/2, d) with the column
+ * position; inside a half, adjacent pair (2i, 2i+1) rotates by
+ * pos * rope_theta^(-2i/(d/2)).
+ *
+ * RMSNorm: y = x / sqrt(mean_c(x^2) + eps) * w[c], per (b, t, h), fp32 math.
+ * q_norm_w / k_norm_w are device pointers to d fp32 weights, or NULL for 1.0.
+ */
+typedef struct {
+  int img_h, img_w;        /* noisy-target latent grid; N_img must equal img_h * img_w */
+  int ref_h, ref_w;        /* reference grid; N_ref must equal ref_h * ref_w (0 x 0 = none) */
+  int ref_row_offset;      /* row shift of the reference grid (e.g. img_h) */
+  float rope_theta;        /* RoPE base, > 0 (workloads: 10000) */
+  float eps;               /* RMSNorm epsilon, >= 0 (workloads: 1e-6) */
+  const float* q_norm_w;   /* [d] fp32 device pointer or NULL */
+  const float* k_norm_w;   /* [d] fp32 device pointer or NULL */
+} jattn_prologue_params;
+
+/*
+ * jattn_prologue — RMSNorm + 2-D RoPE of Q and K, optional E4M3 quantisation.
+ *
+ * Source: the QKV-epilogue fusion of query/key normalisation and rotary
+ * position embedding ("GEMM kernel optimization" section of the tutorial),
+ * and the FP8 Q/K/V attention inputs ("Quantized and sparse attention").
+ *
+ * q, k, v : bf16 [B, N, H, d] inputs (v is read only in mode FP8).
+ * mode JATTN_PROLOGUE_BF16:
+ *   q_out, k_out : bf16 [B, N, H, d]; may equal q, k (in place);
+ *   v_out, *_scale : ignored (may be NULL).
+ * mode JATTN_PROLOGUE_FP8:
+ *   q_out, k_out, v_out : E4M3FN codes, 1 byte each, [B, N, H, d];
+ *   q_scale, k_scale, v_scale : fp32 [B, H, ceil(N / 64)].
+ *   Per (b, h, 64-token block j): amax = max |x| over the block's tokens
+ *   and all d channels of the bf16-rounded Q' (resp. K', V);
+ *   code = E4M3_RNE_satfinite(x * (448 / amax)), scale = amax / 448, both
+ *   fp32 operations correctly rounded; an all-zero block has scale 1 and
+ *   zero codes.  The value a code stands for is decode(code) * scale.
+ * Sizes: B, H >= 1; d == 128 (else UNSUPPORTED); N = N_txt + N_img + N_ref
+ * >= 1; p must be non-NULL and consistent with N_img / N_ref.
+ * All tensor pointers must be 16-byte aligned (else MISALIGNED).
+ */
+JATTN_API int jattn_prologue(const void* q, const void* k, const void* v,
+                   void* q_out, void* k_out, void* v_out,
+                   float* q_scale, float* k_scale, float* v_scale,
+                   int B, int H, int N_txt, int N_img, int N_ref, int d, int mode,
+                   const jattn_prologue_params* p, void* cuda_stream);
+
+/*
+ * jattn_fwd_bf16 — joint attention forward, BF16 operands.
+ *
+ * Source: the VANILLA BF16 attention the tutorial's "Quantized and sparse
+ * attention" section names as the dominant DiT cost at 2048^2; the joint
+ * sequence from "FLUX 3 inference with TensorRT LLM VisualGen".
+ *
+ * q, k, v : bf16 [B, N, H, d] (Q', K' as the prologue writes them).
+ * o       : bf16 [B, N, H, d] output, O = softmax(softmax_scale * Q K^T) V,
+ *           every query against all N keys of its (b, h).
+ * lse     : optional fp32 [B, H, N] output, ln sum_j exp(scale * q.k_j);
+ *           NULL skips it.
+ * The stream split (N_txt / N_img / N_ref) is validated (each >= 0, sum
+ * >= 1) but does not change the result: the sequence is attended as one.
+ * d must be 128; softmax_scale must be finite and > 0.
+ * o must not overlap q, k or v.
+ */
+JATTN_API int jattn_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int H, int N_txt, int N_img, int N_ref, int d,
+                   float softmax_scale, void* cuda_stream);
+
+/*
+ * jattn_fwd_fp8 — joint attention forward from E4M3 block-quantised inputs.
+ *
+ * Source: FP8 Q/K and FP8 V attention ("Quantized and sparse attention"
+ * section of the tutorial, qk_dtype / v_dtype fp8).
+ *
+ * q8, k8, v8 : E4M3FN codes [B, N, H, d] as jattn_prologue(mode FP8) writes.
+ * q_scale, k_scale, v_scale : fp32 [B, H, ceil(N / 64)] block scales.
+ * Computes O = softmax(softmax_scale * Qd Kd^T) Vd with Xd the dequantised
+ * values decode(code) * scale.  QK^T runs on E4M3 operands with fp32
+ * accumulation and the block scales applied to the fp32 scores; P.V runs
+ * with P in FP16 and V's codes widened to FP16 (exact).
+ * o : bf16 [B, N, H, d]; lse : optional fp32 [B, H, N].
+ */
+JATTN_API int jattn_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                  const float* q_scale, const float* k_scale, const float* v_scale,
+                  void* o, float* lse,
+                  int B, int H, int N_txt, int N_img, int N_ref, int d,
+                  float softmax_scale, void* cuda_stream);
+
+/* Human-readable name of a jattn_status value (static string, never NULL). */
+JATTN_API const char* jattn_status_string(int status);
+
+/*
+ * jattn_device_status — synchronise `cuda_stream`, read and clear the device
+ * error word the kernels set when a bounded wait runs out.  Returns JATTN_OK,
+ * JATTN_ERR_TIMEOUT, or JATTN_ERR_CUDA if the synchronisation itself failed.
+ * A diagnostic call: it blocks the host and must not be stream-captured.
+ */
+JATTN_API int jattn_device_status(void* cuda_stream);
+
+/*
+ * jattn_selftest_wait_timeout — launch one CTA that waits, with the same
+ * bounded wait the attention kernels use, on a barrier nothing will ever
+ * complete, for at most `timeout_ns` nanoseconds (1 .. 1e9), then returns.
+ * Exercises the timeout path without a fault or a hang: afterwards
+ * jattn_device_status() must report JATTN_ERR_TIMEOUT.
+ */
+JATTN_API int jattn_selftest_wait_timeout(long long timeout_ns, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JATTN_H_ */

@@ -254,22 +254,20 @@ def joint_attention(q, k, v, scale: float, rows=None):
     ``len(rows)`` rows.  Returns ``O [B, R, H, d]`` float64 and the
     log-sum-exp ``L [B, H, R]`` = ln sum_j exp(scale * q.k_j).
     """
-    q = np.asarray(q, dtype=np.float64)
-    k = np.asarray(k, dtype=np.float64)
-    v = np.asarray(v, dtype=np.float64)
     B, N, H, d = q.shape
     idx = np.arange(N) if rows is None else np.asarray(rows)
     R = len(idx)
     out = np.empty((B, R, H, v.shape[-1]), dtype=np.float64)
     lse = np.empty((B, H, R), dtype=np.float64)
     sc = float(scale)
+    f64 = lambda a: np.asarray(a, dtype=np.float64)   # widen one (b, h) slice at a time
     for b in range(B):
         for h in range(H):
-            s = sc * (q[b, idx, h, :] @ k[b, :, h, :].T)          # [R, N]
+            s = sc * (f64(q[b, idx, h, :]) @ f64(k[b, :, h, :]).T)   # [R, N]
             m = np.max(s, axis=1, keepdims=True)
             p = np.exp(s - m)
             l = np.sum(p, axis=1, keepdims=True)
-            out[b, :, h, :] = (p / l) @ v[b, :, h, :]
+            out[b, :, h, :] = (p / l) @ f64(v[b, :, h, :])
             lse[b, h, :] = (m + np.log(l))[:, 0]
     return out, lse
 

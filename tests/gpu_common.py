@@ -1,0 +1,92 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the
+C-ABI binding, run the oracle on the same seeded inputs, compare."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as O
+from diffusion_transformer_joint_dit_b200 import binding as J
+from diffusion_transformer_joint_dit_b200 import inputs as I
+
+# Tolerances (workload definition): BF16 attention relative L2 <= 5e-3 and
+# max-abs <= 2e-2 on N(0,1) inputs; FP8 attention relative L2 <= 1e-2 against
+# the oracle that applies the same E4M3 block quantisation.
+BF16_REL_L2 = 5e-3
+BF16_MAX_ABS = 2e-2
+FP8_REL_L2 = 1e-2
+
+
+def rel_l2(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    """bf16 / fp32 torch tensor (any device) -> float32 numpy (exact)."""
+    return t.detach().float().cpu().numpy()
+
+
+def prologue_params(w: I.Workload):
+    return J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps)
+
+
+def gpu_prologue_bf16(w: I.Workload, q, k):
+    qd, kd = q.cuda(), k.cuda()
+    qo, ko = torch.empty_like(qd), torch.empty_like(kd)
+    J.jattn_prologue(qd, kd, None, qo, ko, None, None, None, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref,
+                     w.d, J.JATTN_PROLOGUE_BF16, prologue_params(w))
+    torch.cuda.synchronize()
+    return qo, ko
+
+
+def gpu_prologue_fp8(w: I.Workload, q, k, v):
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    shape = (w.B, w.N, w.H, w.d)
+    nblk = -(-w.N // J.JATTN_FP8_BLOCK)
+    q8, k8, v8 = (torch.empty(shape, dtype=torch.uint8, device="cuda") for _ in range(3))
+    qs, ks, vs = (torch.empty((w.B, w.H, nblk), dtype=torch.float32, device="cuda") for _ in range(3))
+    J.jattn_prologue(qd, kd, vd, q8, k8, v8, qs, ks, vs, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+                     J.JATTN_PROLOGUE_FP8, prologue_params(w))
+    torch.cuda.synchronize()
+    return (q8, k8, v8), (qs, ks, vs)
+
+
+def gpu_attn_bf16(w: I.Workload, q, k, v, with_lse: bool = True):
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o = torch.full_like(qd, float("nan"))
+    lse = torch.full((w.B, w.H, w.N), float("nan"), dtype=torch.float32, device="cuda") if with_lse else None
+    J.jattn_fwd_bf16(qd, kd, vd, o, lse, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d, w.softmax_scale)
+    torch.cuda.synchronize()
+    assert J.jattn_device_status() == J.JATTN_OK
+    return o, lse
+
+
+def oracle_prologue_bf16(w: I.Workload, q, k):
+    """Oracle Q', K' (float64) and their bf16 roundings (float64 arrays)."""
+    qp, kp = O.prologue(to_np(q), to_np(k), n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w,
+                        ref_h=w.ref_h, ref_w=w.ref_w, ref_row_offset=w.ref_row_offset,
+                        theta=w.theta, eps=w.eps)
+    return qp, kp, O.bf16_round(qp), O.bf16_round(kp)
+
+
+def check_attention(w: I.Workload, out, lse, q_np, k_np, v_np, rows=None, rel_tol=BF16_REL_L2,
+                    abs_tol=BF16_MAX_ABS, lse_tol=2e-3):
+    """Compare GPU O (and LSE) with the oracle on `rows` (all if None)."""
+    ref, ref_lse = O.joint_attention(q_np, k_np, v_np, w.softmax_scale, rows=rows)
+    o = to_np(out)
+    if rows is not None:
+        o = o[:, rows]
+    assert np.isfinite(o).all(), "unwritten or non-finite output"
+    err = rel_l2(o, ref)
+    mx = float(np.max(np.abs(o - ref)))
+    assert err <= rel_tol, f"rel-L2 {err:.3e} > {rel_tol}"
+    assert mx <= abs_tol, f"max-abs {mx:.3e} > {abs_tol}"
+    if lse is not None:
+        l = to_np(lse)
+        if rows is not None:
+            l = l[:, :, rows]
+        assert np.max(np.abs(l - ref_lse)) <= lse_tol
+    return err, mx

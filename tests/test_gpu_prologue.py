@@ -1,0 +1,92 @@
+"""GPU parity of jattn_prologue against the float64 oracle.
+
+BF16 mode: every output element within 1 bf16 ulp of the oracle's value
+rounded to bf16 (the kernel works in fp32), and at least 99.9% identical.
+FP8 mode: E4M3 codes at least 99.99% identical to the oracle's quantisation
+of its own bf16-rounded Q', K' (and of V), every mismatch one code step
+apart; block scales identical wherever the block maxima agree.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from diffusion_transformer_joint_dit_b200 import binding as J
+from diffusion_transformer_joint_dit_b200 import inputs as I
+from tests.gpu_common import (gpu_prologue_bf16, gpu_prologue_fp8, oracle_prologue_bf16, prologue_params,
+                              to_np)
+
+pytestmark = pytest.mark.gpu
+
+EDGE = {
+    "i2i_small": I.custom("i2i_small", B=2, H=3, n_txt=8, img_h=4, img_w=4, ref_h=4, ref_w=4, ref_row_offset=4),
+    "text_only_1": I.custom("text_only_1", B=1, H=1, n_txt=1, img_h=0, img_w=0),
+    "rect_grid": I.custom("rect_grid", B=1, H=5, n_txt=3, img_h=7, img_w=13, ref_h=2, ref_w=9, ref_row_offset=7),
+    "tail_block": I.custom("tail_block", B=1, H=2, n_txt=70, img_h=0, img_w=0),
+}
+
+
+def _bf16_close(got, ref):
+    d = O.bf16_ulp_distance(to_np(got), ref)
+    assert d.max() <= 1, f"max ulp distance {d.max()}"
+    assert (d == 0).mean() >= 0.999, f"identical fraction {(d == 0).mean():.5f}"
+
+
+@pytest.mark.parametrize("name", ["tiny", "t2i_1024", "i2i_small", "text_only_1", "rect_grid", "tail_block"])
+def test_prologue_bf16_matches_oracle(cuda_ok, name):
+    w = I.WORKLOADS.get(name) or EDGE[name]
+    q, k, _ = I.make_qkv(w, seed=3)
+    qo, ko = gpu_prologue_bf16(w, q, k)
+    _, _, qb, kb = oracle_prologue_bf16(w, q, k)
+    _bf16_close(qo, qb)
+    _bf16_close(ko, kb)
+
+
+def test_prologue_bf16_in_place_and_weights(cuda_ok):
+    w = EDGE["i2i_small"]
+    q, k, _ = I.make_qkv(w, seed=4)
+    rng = np.random.default_rng(5)
+    wq = rng.uniform(0.5, 1.5, 128).astype(np.float32)
+    wk = rng.uniform(0.5, 1.5, 128).astype(np.float32)
+    qd, kd = q.cuda(), k.cuda()
+    wqd, wkd = torch.from_numpy(wq).cuda(), torch.from_numpy(wk).cuda()
+    p = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps,
+                               q_norm_w=wqd, k_norm_w=wkd)
+    J.jattn_prologue(qd, kd, None, qd, kd, None, None, None, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+                     J.JATTN_PROLOGUE_BF16, p)
+    torch.cuda.synchronize()
+    qp, kp = O.prologue(to_np(q), to_np(k), n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w, ref_h=w.ref_h,
+                        ref_w=w.ref_w, ref_row_offset=w.ref_row_offset, theta=w.theta, eps=w.eps,
+                        q_norm_w=wq, k_norm_w=wk)
+    _bf16_close(qd, O.bf16_round(qp))
+    _bf16_close(kd, O.bf16_round(kp))
+
+
+def _codes_close(got, ref):
+    got = got.cpu().numpy()
+    same = got == ref
+    frac = same.mean()
+    assert frac >= 0.9999, f"identical code fraction {frac:.6f}"
+    if not same.all():
+        g, r = got[~same].astype(np.int64), ref[~same].astype(np.int64)
+        assert ((g & 0x80) == (r & 0x80)).all() and (np.abs((g & 0x7F) - (r & 0x7F)) == 1).all()
+
+
+def _scales_close(got, ref):
+    got = got.cpu().numpy()
+    rel = np.abs(got.astype(np.float64) / ref - 1.0)
+    assert rel.max() <= 2.0 ** -7, f"scale rel diff {rel.max():.3e}"
+    assert (got == ref).mean() >= 0.99
+
+
+@pytest.mark.parametrize("name", ["tiny", "i2i_small", "tail_block", "rect_grid", "t2i_2048_fp8"])
+def test_prologue_fp8_matches_oracle(cuda_ok, name):
+    w = I.WORKLOADS.get(name) or EDGE[name]
+    q, k, v = I.make_qkv(w, seed=6)
+    (q8, k8, v8), (qs, ks, vs) = gpu_prologue_fp8(w, q, k, v)
+    _, _, qb, kb = oracle_prologue_bf16(w, q, k)
+    for got_c, got_s, x in ((q8, qs, qb), (k8, ks, kb), (v8, vs, to_np(v))):
+        codes, scales = O.block_quantize_e4m3(x.astype(np.float32))
+        _codes_close(got_c, codes)
+        _scales_close(got_s, scales)
