@@ -28,13 +28,17 @@ JATTN_PROLOGUE_FP8 = 1
 JATTN_FP8_BLOCK = 64
 
 EXPORTED = ("jattn_prologue", "jattn_fwd_bf16", "jattn_fwd_fp8", "jattn_status_string",
-            "jattn_device_status", "jattn_selftest_wait_timeout")
+            "jattn_device_status", "jattn_selftest_wait_timeout", "jattn_selftest_exp2_poly",
+            "jattn_last_cuda_error")
 
 
 class JattnError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {status_name(status)} ({status})")
+        msg = f"{fn} failed: {status_name(status)} ({status})"
+        if status == JATTN_ERR_CUDA:
+            msg += f" [{jattn_last_cuda_error()}]"
+        super().__init__(msg)
 
 
 class jattn_prologue_params(ctypes.Structure):
@@ -74,6 +78,10 @@ def load_library():
     lib.jattn_device_status.restype = _I
     lib.jattn_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _P]
     lib.jattn_selftest_wait_timeout.restype = _I
+    lib.jattn_selftest_exp2_poly.argtypes = [_P, _P, _I, _P]
+    lib.jattn_selftest_exp2_poly.restype = _I
+    lib.jattn_last_cuda_error.argtypes = []
+    lib.jattn_last_cuda_error.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
@@ -146,6 +154,10 @@ def jattn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B: int, H: int,
     return st
 
 
+def jattn_last_cuda_error() -> str:
+    return load_library().jattn_last_cuda_error().decode()
+
+
 def jattn_device_status(stream=None) -> int:
     return load_library().jattn_device_status(_stream(stream))
 
@@ -154,4 +166,11 @@ def jattn_selftest_wait_timeout(timeout_ns: int, stream=None, *, check: bool = T
     st = load_library().jattn_selftest_wait_timeout(int(timeout_ns), _stream(stream))
     if check:
         _check("jattn_selftest_wait_timeout", st)
+    return st
+
+
+def jattn_selftest_exp2_poly(x, y, n: int, stream=None, *, check: bool = True) -> int:
+    st = load_library().jattn_selftest_exp2_poly(_ptr(x), _ptr(y), int(n), _stream(stream))
+    if check:
+        _check("jattn_selftest_exp2_poly", st)
     return st

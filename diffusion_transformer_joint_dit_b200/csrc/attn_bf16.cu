@@ -33,6 +33,7 @@
 // query rows read zero-filled Q and are not stored.
 #include "jattn_internal.h"
 #include "sm100_ptx.cuh"
+#include "softmax_sm100.cuh"
 
 namespace jattn {
 
@@ -51,6 +52,7 @@ constexpr int kMmaWarp = kSoftmaxWarps + 1;    // 9
 constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kPolyEvery = 4;     // 1 pair in 4 takes the polynomial exp2 (25%)
 
 struct Ctrl {
   uint64_t q_full;
@@ -276,15 +278,9 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i >= nvalid) sv[c][i] = __float_as_uint(-INFINITY);
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        mx0 = fmaxf(mx0, __uint_as_float(sv[0][i]));
-        mx1 = fmaxf(mx1, __uint_as_float(sv[1][i]));
-        mx2 = fmaxf(mx2, __uint_as_float(sv[2][i]));
-        mx3 = fmaxf(mx3, __uint_as_float(sv[3][i]));
-      }
-      const float mnew = fmaxf(m, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2);
+      float mx_lo, mx_hi;
+      row_max_halves(sv, mx_lo, mx_hi);
+      const float mnew = fmaxf(m, fmaxf(mx_lo, mx_hi) * sl2);
       const bool need = mnew > m + kRescaleThreshold;
       float corr = 1.f;
       if (need) {
@@ -292,6 +288,16 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         l *= corr;
         m = mnew;
       }
+      // P = exp2(s * scale * log2e - m), packed two bf16 per 32-bit word in
+      // place: keys [0,64) land in sv[0], keys [64,128) in sv[2].  Full
+      // tiles send a quarter of the pairs through the polynomial exp2.
+      float l0, l1;
+      exp_pack_tile<false, kPolyEvery>(sv, sl2, -m, sl2, -m, nvalid >= kBN, l0, l1);
+      l += l0 + l1;
+      tmem_st32(s_addr, sv[0]);
+      tmem_st32(s_addr + 32, sv[2]);
+      // O correction after P is out of registers (keeps register pressure
+      // down); it only has to land before this tile's P.V is issued.
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -303,25 +309,6 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           tmem_st32(o_addr + c * 32, ov);
         }
       }
-      // P = exp2(x - m), packed two bf16 per 32-bit word in place: keys
-      // [0,64) land in sv[0], keys [64,128) in sv[2] (each packed word is
-      // written at or before the index it was read from).
-      const float neg_m = -m;
-      float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c][i]), sl2, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c][i + 1]), sl2, neg_m));
-          l0 += p0;
-          l1 += p1;
-          sv[c & 2][(c & 1) * 16 + (i >> 1)] = pack_bf16x2(p0, p1);
-        }
-      }
-      l += l0 + l1;
-      tmem_st32(s_addr, sv[0]);
-      tmem_st32(s_addr + 32, sv[2]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctrl->p_full[t]);
@@ -384,7 +371,7 @@ cudaError_t launch_attn_bf16(const AttnProblem& p, cudaStream_t s) {
   prm.timeout_ns = p.timeout_ns;
   dim3 grid((p.N + kBM * kTiles - 1) / (kBM * kTiles), p.H, p.B);
   attn_bf16_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, prm);
-  return cudaPeekAtLastError();
+  return cudaGetLastError();
 }
 
 }  // namespace jattn

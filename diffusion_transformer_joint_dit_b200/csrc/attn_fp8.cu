@@ -25,6 +25,7 @@
 
 #include "jattn_internal.h"
 #include "sm100_ptx.cuh"
+#include "softmax_sm100.cuh"
 
 namespace jattn {
 
@@ -47,6 +48,7 @@ constexpr int kCvtThreads = 64;
 constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // 384
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kPolyEvery = 4;     // 1 pair in 4 takes the polynomial exp2 (25%)
 
 struct Ctrl {
   uint64_t q_full;
@@ -354,18 +356,12 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i >= nvalid) sv[c][i] = __float_as_uint(-INFINITY);
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        mx0 = fmaxf(mx0, __uint_as_float(sv[0][i]));
-        mx1 = fmaxf(mx1, __uint_as_float(sv[1][i]));
-        mx2 = fmaxf(mx2, __uint_as_float(sv[2][i]));
-        mx3 = fmaxf(mx3, __uint_as_float(sv[3][i]));
-      }
+      float mx_lo, mx_hi;
+      row_max_halves(sv, mx_lo, mx_hi);
       // Scaled maxima of the two halves (scales are > 0; a fully masked
       // half has max -inf and stays -inf).
-      const float hm0 = fmaxf(mx0, mx1) * c0;
-      const float hm1 = fmaxf(mx2, mx3) * c1;
+      const float hm0 = mx_lo * c0;
+      const float hm1 = mx_hi * c1;
       const float mnew = fmaxf(m, fmaxf(hm0, hm1));
       const bool need = mnew > m + kRescaleThreshold;
       float corr = 1.f;
@@ -374,6 +370,17 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         l *= corr;
         m = mnew;
       }
+      // Exponent biases fold the V block scales: P' = P * sv / 2^e.
+      const float bias0 = __log2f(sv0) - lg_norm - m;
+      const float bias1 = __log2f(sv1) - lg_norm - m;
+      float l0, l1;
+      exp_pack_tile<true, kPolyEvery>(sv, c0, bias0, c1, bias1, nvalid >= kBN, l0, l1);
+      // Undo the V-scale fold for the row sum: sum P = sum P' * 2^e / sv.
+      l += l0 * (v_norm / sv0) + (nvalid > 64 ? l1 * (v_norm / sv1) : 0.f);
+      tmem_st32(s_addr, sv[0]);
+      tmem_st32(s_addr + 32, sv[2]);
+      // O correction after P is out of registers (keeps register pressure
+      // down); it only has to land before this tile's P.V is issued.
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -385,28 +392,6 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tmem_st32(o_addr + c * 32, ov);
         }
       }
-      // Exponent biases fold the V block scales: P' = P * sv / 2^e.
-      const float bias0 = __log2f(sv0) - lg_norm - m;
-      const float bias1 = __log2f(sv1) - lg_norm - m;
-      float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float cc = c < 2 ? c0 : c1;
-        const float bb = c < 2 ? bias0 : bias1;
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c][i]), cc, bb));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c][i + 1]), cc, bb));
-          acc += p0 + p1;
-          sv[c & 2][(c & 1) * 16 + (i >> 1)] = pack_f16x2(p0, p1);
-        }
-        if (c < 2) l0 += acc; else l1 += acc;
-      }
-      // Undo the V-scale fold for the row sum: sum P = sum P' * 2^e / sv.
-      l += l0 * (v_norm / sv0) + (nvalid > 64 ? l1 * (v_norm / sv1) : 0.f);
-      tmem_st32(s_addr, sv[0]);
-      tmem_st32(s_addr + 32, sv[2]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctrl->p_full[t]);
@@ -472,7 +457,7 @@ cudaError_t launch_attn_fp8(const AttnProblem& p, cudaStream_t s) {
   prm.timeout_ns = p.timeout_ns;
   dim3 grid((p.N + kBM * kTiles - 1) / (kBM * kTiles), p.H, p.B);
   attn_fp8_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, prm);
-  return cudaPeekAtLastError();
+  return cudaGetLastError();
 }
 
 }  // namespace jattn

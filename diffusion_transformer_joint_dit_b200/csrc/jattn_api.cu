@@ -51,9 +51,26 @@ __global__ void wait_selftest_kernel(uint64_t timeout_ns) {
   __syncthreads();
 }
 
+// Polynomial-exp2 self test: pairs of inputs through the softmax's helper.
+__global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i];
+  const float b = i + 1 < n ? x[i + 1] : 0.f;
+  const uint64_t r = exp2_poly2(f2_pack(a, b));
+  y[i] = f2_lo(r);
+  if (i + 1 < n) y[i + 1] = f2_hi(r);
+}
+
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
 
-int map_err(cudaError_t e) { return e == cudaSuccess ? JATTN_OK : JATTN_ERR_CUDA; }
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+int map_err(cudaError_t e) {
+  if (e == cudaSuccess) return JATTN_OK;
+  t_last_cuda_error = e;
+  return JATTN_ERR_CUDA;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -113,7 +130,7 @@ cudaError_t set_smem_attr(const void* func, int bytes) {
 
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t s) {
   wait_selftest_kernel<<<1, 32, 0, s>>>(timeout_ns);
-  return cudaPeekAtLastError();
+  return cudaGetLastError();
 }
 
 }  // namespace jattn
@@ -218,13 +235,16 @@ int jattn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q
   return map_err(e);
 }
 
+const char* jattn_last_cuda_error(void) { return cudaGetErrorName(t_last_cuda_error); }
+
 int jattn_device_status(void* cuda_stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return JATTN_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return map_err(e);
   unsigned int word = 0;
-  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return JATTN_ERR_CUDA;
+  if ((e = cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word))) != cudaSuccess) return map_err(e);
   if (word != 0) {
     const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return JATTN_ERR_CUDA;
+    if ((e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero))) != cudaSuccess) return map_err(e);
     return JATTN_ERR_TIMEOUT;
   }
   return JATTN_OK;
@@ -233,6 +253,14 @@ int jattn_device_status(void* cuda_stream) {
 int jattn_selftest_wait_timeout(long long timeout_ns, void* cuda_stream) {
   if (timeout_ns < 1 || timeout_ns > 1000000000ll) return JATTN_ERR_INVALID_ARG;
   return map_err(launch_wait_selftest(static_cast<uint64_t>(timeout_ns), static_cast<cudaStream_t>(cuda_stream)));
+}
+
+int jattn_selftest_exp2_poly(const float* x, float* y, int n, void* cuda_stream) {
+  if (x == nullptr || y == nullptr || n < 1) return JATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 7u) return JATTN_ERR_MISALIGNED;
+  const int pairs = (n + 1) / 2;
+  exp2_poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(x, y, n);
+  return map_err(cudaGetLastError());
 }
 
 }  // extern "C"

@@ -313,13 +313,13 @@ cudaError_t launch_prologue_bf16(const PrologueArgs& a, cudaStream_t s) {
   const long long tokens = static_cast<long long>(a.B) * a.N;
   const unsigned grid = static_cast<unsigned>((tokens + kBf16Warps - 1) / kBf16Warps);
   prologue_bf16_kernel<<<grid, kBf16Warps * 32, 0, s>>>(a);
-  return cudaPeekAtLastError();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_prologue_fp8(const PrologueArgs& a, cudaStream_t s) {
   dim3 grid((a.N + kQuantBlock - 1) / kQuantBlock, (a.H + kFp8Heads - 1) / kFp8Heads, a.B);
   prologue_fp8_kernel<<<grid, kFp8Warps * 32, 0, s>>>(a);
-  return cudaPeekAtLastError();
+  return cudaGetLastError();
 }
 
 }  // namespace jattn

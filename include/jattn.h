@@ -34,7 +34,8 @@
  *
  * Errors.  Arguments are checked before any launch; a rejected call launches
  * nothing and returns a jattn_status below.  After a launch the return is the
- * launch status (cudaPeekAtLastError) mapped to JATTN_ERR_CUDA.  Every wait
+ * launch status (cudaGetLastError, which also clears a pending non-sticky
+ * error of the calling thread) mapped to JATTN_ERR_CUDA.  Every wait
  * inside the attention kernels is bounded; a wait that runs out sets a device
  * error word and the kernel returns early, leaving its outputs undefined;
  * jattn_device_status() reports and clears it.
@@ -166,6 +167,13 @@ JATTN_API int jattn_fwd_fp8(const void* q8, const void* k8, const void* v8,
 JATTN_API const char* jattn_status_string(int status);
 
 /*
+ * jattn_last_cuda_error — name of the CUDA runtime error behind the last
+ * JATTN_ERR_CUDA returned on the calling thread ("cudaSuccess" if none).
+ * Static string, never NULL.
+ */
+JATTN_API const char* jattn_last_cuda_error(void);
+
+/*
  * jattn_device_status — synchronise `cuda_stream`, read and clear the device
  * error word the kernels set when a bounded wait runs out.  Returns JATTN_OK,
  * JATTN_ERR_TIMEOUT, or JATTN_ERR_CUDA if the synchronisation itself failed.
@@ -181,6 +189,15 @@ JATTN_API int jattn_device_status(void* cuda_stream);
  * jattn_device_status() must report JATTN_ERR_TIMEOUT.
  */
 JATTN_API int jattn_selftest_wait_timeout(long long timeout_ns, void* cuda_stream);
+
+/*
+ * jattn_selftest_exp2_poly — evaluate, for n floats x (device pointers), the
+ * range-reduced polynomial exp2 the attention softmax uses for part of its
+ * exponentials, writing y[i] ~ 2^x[i].  Lets tests check its error bound
+ * (relative 7.5e-5 from the degree-3 minimax fit, for x in [-126, 8]).
+ * n >= 1; x and y 8-byte aligned; asynchronous on cuda_stream.
+ */
+JATTN_API int jattn_selftest_exp2_poly(const float* x, float* y, int n, void* cuda_stream);
 
 #ifdef __cplusplus
 }

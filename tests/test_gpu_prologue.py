@@ -1,7 +1,12 @@
 """GPU parity of jattn_prologue against the float64 oracle.
 
-BF16 mode: every output element within 1 bf16 ulp of the oracle's value
-rounded to bf16 (the kernel works in fp32), and at least 99.9% identical.
+BF16 mode: the kernel works in fp32, so its value y differs from the exact
+(float64) oracle value y* by the fp32 rounding of the norm and rotation,
+at most about 2^-20 times the norm of the rotated channel pair.  Every
+element must satisfy |y - y*| <= ulp_bf16(y*) + 2^-18 * |pair|; at least
+99.99% must be within one bf16 code point of y* rounded to bf16 and at
+least 99.9% identical to it.  (Near-zero outputs of a rotation lose their
+relative accuracy by cancellation, so a pure ulp bound would not hold.)
 FP8 mode: E4M3 codes at least 99.99% identical to the oracle's quantisation
 of its own bf16-rounded Q', K' (and of V), every mismatch one code step
 apart; block scales identical wherever the block maxima agree.
@@ -27,9 +32,16 @@ EDGE = {
 }
 
 
-def _bf16_close(got, ref):
-    d = O.bf16_ulp_distance(to_np(got), ref)
-    assert d.max() <= 1, f"max ulp distance {d.max()}"
+def _bf16_close(got, exact):
+    g = to_np(got).astype(np.float64)
+    ref = O.bf16_round(exact)
+    pair = np.sqrt(exact[..., 0::2] ** 2 + exact[..., 1::2] ** 2).repeat(2, axis=-1)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
+    bound = ulp + 2.0 ** -18 * pair
+    worst = np.max(np.abs(g - exact) - bound)
+    assert worst <= 0, f"error exceeds bound by {worst:.3e}"
+    d = O.bf16_ulp_distance(g, ref)
+    assert (d <= 1).mean() >= 0.9999, f"within-1-ulp fraction {(d <= 1).mean():.6f}"
     assert (d == 0).mean() >= 0.999, f"identical fraction {(d == 0).mean():.5f}"
 
 
@@ -38,9 +50,9 @@ def test_prologue_bf16_matches_oracle(cuda_ok, name):
     w = I.WORKLOADS.get(name) or EDGE[name]
     q, k, _ = I.make_qkv(w, seed=3)
     qo, ko = gpu_prologue_bf16(w, q, k)
-    _, _, qb, kb = oracle_prologue_bf16(w, q, k)
-    _bf16_close(qo, qb)
-    _bf16_close(ko, kb)
+    qp, kp, _, _ = oracle_prologue_bf16(w, q, k)
+    _bf16_close(qo, qp)
+    _bf16_close(ko, kp)
 
 
 def test_prologue_bf16_in_place_and_weights(cuda_ok):
@@ -59,8 +71,8 @@ def test_prologue_bf16_in_place_and_weights(cuda_ok):
     qp, kp = O.prologue(to_np(q), to_np(k), n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w, ref_h=w.ref_h,
                         ref_w=w.ref_w, ref_row_offset=w.ref_row_offset, theta=w.theta, eps=w.eps,
                         q_norm_w=wq, k_norm_w=wk)
-    _bf16_close(qd, O.bf16_round(qp))
-    _bf16_close(kd, O.bf16_round(kp))
+    _bf16_close(qd, qp)
+    _bf16_close(kd, kp)
 
 
 def _codes_close(got, ref):
