@@ -176,7 +176,9 @@ def e4m3_encode(v) -> np.ndarray:
     Written from the definition of round-to-nearest-even on the finite
     value set: clamp |v| to 448 ("satfinite"), pick the nearest of the 127
     non-negative finite values, and on an exact tie take the code whose
-    last mantissa bit is 0.  Sign is carried separately; NaN maps to 0x7F.
+    last mantissa bit is 0.  The sign bit is carried separately and kept
+    when the magnitude rounds to zero (a negative value gives -0, code
+    0x80, as IEEE rounding does); NaN maps to 0x7F.
     """
     v = np.asarray(v, dtype=np.float64)
     a = np.minimum(np.abs(v), E4M3_MAX)
@@ -186,7 +188,7 @@ def e4m3_encode(v) -> np.ndarray:
     d_lo = a - _POS_VALUES[lo]
     pick_lo = (d_lo < d_hi) | ((d_lo == d_hi) & ((_POS_CODES[lo] & 1) == 0))
     code = np.where(pick_lo, _POS_CODES[lo], _POS_CODES[hi])
-    code = np.where(np.signbit(v) & (code != 0), code | 0x80, code)
+    code = np.where(np.signbit(v), code | 0x80, code)
     code = np.where(np.isnan(v), 0x7F, code)
     return code.astype(np.uint8)
 

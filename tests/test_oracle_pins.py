@@ -206,9 +206,7 @@ def test_e4m3_encode_against_torch_cast():
     v = np.clip(v, -448, 448)
     ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     mine = O.e4m3_encode(v)
-    # torch keeps -0 for tiny negatives; the oracle maps them to +0 (same value)
-    same = (mine == ref) | ((O.e4m3_decode(mine) == 0) & (O.e4m3_decode(ref) == 0))
-    assert same.all()
+    assert np.array_equal(mine, ref)                     # including -0 (0x80) for tiny negatives
 
 
 def test_e4m3_ties_and_saturation():
@@ -218,10 +216,12 @@ def test_e4m3_ties_and_saturation():
     assert O.e4m3_encode(464.0) == 0x7E
     assert O.e4m3_encode(1e6) == 0x7E
     assert O.e4m3_encode(-1e6) == 0xFE
+    assert O.e4m3_encode(-2.0 ** -12) == 0x80      # rounds to zero, keeps the sign
+    assert O.e4m3_encode(-0.0) == 0x80 and O.e4m3_encode(0.0) == 0x00
 
 
 def test_e4m3_roundtrip_all_finite_codes():
-    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F and c != 0x80])
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F])   # -0 (0x80) included
     assert np.array_equal(O.e4m3_encode(O.e4m3_decode(codes)), codes)
 
 
