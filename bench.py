@@ -53,6 +53,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU oracle baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-path timing object")
     return ap.parse_args()
 
 
@@ -233,6 +234,60 @@ def run_reference(args, rank: int, world: int):
 
 # -------------------------------------------------------------------- ours ----
 
+def time_fp8_path(J, dev, stream, rank: int, peaks, peaks_src, steps: int = 10):
+    """FP8 path on its own workload (2048^2, no CFG): jattn_prologue in FP8
+    mode (RMSNorm + RoPE + E4M3 block quantisation of Q, K, V) followed by
+    jattn_fwd_fp8.  Reported beside the headline line, not instead of it."""
+    w = I.WORKLOADS["t2i_2048_fp8"]
+    q, k, v = (t.to(dev) for t in I.make_qkv(w, seed=rank))
+    shape = (w.B, w.N, w.H, w.d)
+    nblk = -(-w.N // J.JATTN_FP8_BLOCK)
+    q8, k8, v8 = (torch.empty(shape, dtype=torch.uint8, device=dev) for _ in range(3))
+    qs, ks, vs = (torch.empty((w.B, w.H, nblk), dtype=torch.float32, device=dev) for _ in range(3))
+    o = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    params = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps)
+    h = stream.cuda_stream
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        J.jattn_prologue(q, k, v, q8, k8, v8, qs, ks, vs, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+                         J.JATTN_PROLOGUE_FP8, params, h)
+        if ev is not None:
+            ev[1].record(stream)
+        J.jattn_fwd_fp8(q8, k8, v8, qs, ks, vs, o, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+                        w.softmax_scale, h)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(3):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for e in evs:
+        step(e)
+    torch.cuda.synchronize(dev)
+    if J.jattn_device_status(h) != J.JATTN_OK:
+        raise RuntimeError("device error word set during FP8 timing")
+    pro = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    fp8_peak = 2.0 * peaks["bf16_tflops"]  # nominal dense fp8 : bf16 ratio 2
+    achieved = w.flops / (att * 1e-3) / 1e12
+    pro_bytes = w.B * w.N * w.H * w.d * (3 * 2 + 3 * 1) + 3 * w.B * w.H * nblk * 4
+    return {
+        "workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d}, E4M3 Q/K/V with per-64-token scales",
+        "steps": steps, "attention_ms": att, "prologue_ms": pro,
+        "value": w.flops / ((att + pro) * 1e-3) / 1e12, "unit": UNIT,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp8_peak,
+                     "peak_source": f"{peaks_src} bf16_tflops x 2 (nominal dense fp8/bf16 ratio)",
+                     "bf16_peak_frac": achieved / peaks["bf16_tflops"]},
+        "prologue_roofline": {"bound": "hbm", "achieved": pro_bytes / (pro * 1e-3) / 1e9,
+                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": pro_bytes / (pro * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+    }
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     from diffusion_transformer_joint_dit_b200 import binding as J
 
@@ -358,6 +413,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "gpu_launches": 2 * K,
         "clocks": clocks,
     }
+    if not args.no_fp8:
+        line["fp8_path"] = time_fp8_path(J, dev, stream, rank, peaks, peaks_src)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k_: v_ for k_, v_ in cpu_baseline(w, q, k, v, args.cpu_seconds).items()
                                 if k_ != "seconds"}

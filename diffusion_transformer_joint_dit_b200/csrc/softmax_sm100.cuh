@@ -47,8 +47,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // mantissa bits of t, whose bit pattern shifted left by 23 is n in the
 // exponent field.  p is the degree-3 minimax fit of 2^f (relative error
 // 7.5e-5) computed by fit_exp2_poly.py in this directory.  Arguments below
-// -126 are clamped (the result is then ~1e-38, not 0); callers use it only
-// on unmasked scores, which the lazy-max softmax keeps within [-inf, 8].
+// -125 are clamped (the result is then ~2^-125, not 0, and 2^n p(f) stays a
+// normal float); callers use it only on unmasked scores, which the lazy-max
+// softmax keeps within [-inf, 8].
 constexpr float kPolyC0 = 9.999280572e-01f;
 constexpr float kPolyC1 = 6.932609677e-01f;
 constexpr float kPolyC2 = 2.426111251e-01f;
@@ -56,7 +57,7 @@ constexpr float kPolyC3 = 5.517166853e-02f;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  const float xl = fmaxf(f2_lo(x2), -126.f), xh = fmaxf(f2_hi(x2), -126.f);
+  const float xl = fmaxf(f2_lo(x2), -125.f), xh = fmaxf(f2_hi(x2), -125.f);
   const uint64_t x = f2_pack(xl, xh);
   const uint64_t t = f2_add(x, f2_pack(kRoundMagic, kRoundMagic));
   const uint64_t n = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));
@@ -87,7 +88,7 @@ __device__ __forceinline__ void row_max_halves(const uint32_t (&sv)[4][32], floa
 
 // P = exp2(s * c + b) with (c, b) per 64-key half, packed in place two per
 // word (keys [0,64) into sv[0], [64,128) into sv[2]) as bf16 or fp16, and
-// the fp32 row sums of each half.  With `poly`, one pair in every
+// the fp32 row sums of each half of the packed (rounded) values.  With `poly`, one pair in every
 // kPolyEvery pairs takes the polynomial exp2 instead of MUFU.
 template <bool kF16, int kPolyEvery>
 __device__ __forceinline__ void exp_pack_tile(uint32_t (&sv)[4][32], float c_lo, float b_lo, float c_hi,
@@ -108,9 +109,20 @@ __device__ __forceinline__ void exp_pack_tile(uint32_t (&sv)[4][32], float c_lo,
       } else {
         p = f2_pack(ex2_approx(f2_lo(x)), ex2_approx(f2_hi(x)));
       }
-      acc = f2_add(acc, p);
       const uint32_t packed = kF16 ? pack_f16x2(f2_lo(p), f2_hi(p)) : pack_bf16x2(f2_lo(p), f2_hi(p));
       sv[c & 2][(c & 1) * 16 + (i >> 1)] = packed;
+      // The row sum adds the *rounded* P the MMA multiplies V by, so that
+      // O = sum(P V) / sum(P) uses one set of weights.  With the lazy max a
+      // dominant key's P lies in (1, 2^8] and is inexact in bf16; summing
+      // the rounded value cancels that rounding in the quotient.
+      uint64_t pr;
+      if (kF16) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&packed));
+        pr = f2_pack(f.x, f.y);
+      } else {
+        pr = f2_pack(__uint_as_float(packed << 16), __uint_as_float(packed & 0xFFFF0000u));
+      }
+      acc = f2_add(acc, pr);
     }
     if (c < 2) acc_lo = f2_add(acc_lo, acc); else acc_hi = f2_add(acc_hi, acc);
   }

@@ -194,7 +194,8 @@ JATTN_API int jattn_selftest_wait_timeout(long long timeout_ns, void* cuda_strea
  * jattn_selftest_exp2_poly — evaluate, for n floats x (device pointers), the
  * range-reduced polynomial exp2 the attention softmax uses for part of its
  * exponentials, writing y[i] ~ 2^x[i].  Lets tests check its error bound
- * (relative 7.5e-5 from the degree-3 minimax fit, for x in [-126, 8]).
+ * (relative 7.5e-5 from the degree-3 minimax fit, for x in [-125, 8];
+ * smaller x is clamped to -125).
  * n >= 1; x and y 8-byte aligned; asynchronous on cuda_stream.
  */
 JATTN_API int jattn_selftest_exp2_poly(const float* x, float* y, int n, void* cuda_stream);
