@@ -295,7 +295,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // P = exp2(s * scale * log2e - m), packed two bf16 per 32-bit word in
       // place: keys [0,64) land in sv[0], keys [64,128) in sv[2].
       float l0, l1;
-      exp_pack_tile<false, kPolyEvery>(sv, sl2, -m, sl2, -m, nvalid >= kBN, l0, l1);
+      exp_pack_tile<false, kPolyEvery, true>(sv, sl2, -m, sl2, -m, nvalid >= kBN, l0, l1);
       l += l0 + l1;
       tmem_st32(s_addr, sv[0]);
       tmem_st32(s_addr + 32, sv[2]);

@@ -48,7 +48,10 @@ constexpr int kCvtThreads = 64;
 constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // 384
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
-constexpr int kPolyEvery = 4;     // 1 pair in 4 takes the polynomial exp2 (25%)
+// All exponentials on MUFU: on B200 a 1-in-4 or 1-in-8 polynomial share
+// measured slower (the polynomial's issue slots cost more than the MUFU
+// time it frees at this kernel's register budget).
+constexpr int kPolyEvery = 0;
 
 struct Ctrl {
   uint64_t q_full;
@@ -94,10 +97,6 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint6
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // 16 E4M3 codes -> 16 FP16 values (exact), as two 16-byte chunks.
@@ -299,8 +298,11 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint8_t* dst = smem + kSmemVh + vb * kTile16;
 #pragma unroll 4
       for (int i = 0; i < (kBN * 8) / kCvtThreads; ++i) {
-        const int idx = ct + i * kCvtThreads;  // 16-byte source chunk: row r, chunk c16
-        const int r = idx >> 3, c16 = idx & 7;
+        // 16-byte source chunk (row r, channel chunk c16).  Consecutive lanes
+        // take consecutive rows of one chunk column: each group of 8 lanes
+        // then touches 8 distinct swizzled bank groups on load and store.
+        const int idx = ct + i * kCvtThreads;
+        const int r = idx & (kBN - 1), c16 = idx >> 7;
         const uint4 raw = *reinterpret_cast<const uint4*>(src + r * 128 + ((c16 ^ (r & 7)) << 4));
         uint4 lo, hi;
         widen16(raw, lo, hi);
@@ -374,7 +376,7 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float bias0 = __log2f(sv0) - lg_norm - m;
       const float bias1 = __log2f(sv1) - lg_norm - m;
       float l0, l1;
-      exp_pack_tile<true, kPolyEvery>(sv, c0, bias0, c1, bias1, nvalid >= kBN, l0, l1);
+      exp_pack_tile<true, kPolyEvery, false>(sv, c0, bias0, c1, bias1, nvalid >= kBN, l0, l1);
       // Undo the V-scale fold for the row sum: sum P = sum P' * 2^e / sv.
       l += l0 * (v_norm / sv0) + (nvalid > 64 ? l1 * (v_norm / sv1) : 0.f);
       tmem_st32(s_addr, sv[0]);

@@ -88,9 +88,10 @@ __device__ __forceinline__ void row_max_halves(const uint32_t (&sv)[4][32], floa
 
 // P = exp2(s * c + b) with (c, b) per 64-key half, packed in place two per
 // word (keys [0,64) into sv[0], [64,128) into sv[2]) as bf16 or fp16, and
-// the fp32 row sums of each half of the packed (rounded) values.  With `poly`, one pair in every
+// the fp32 row sums of each half: of the packed (rounded) values when
+// kRoundedSum, else of the fp32 values.  With `poly`, one pair in every
 // kPolyEvery pairs takes the polynomial exp2 instead of MUFU.
-template <bool kF16, int kPolyEvery>
+template <bool kF16, int kPolyEvery, bool kRoundedSum>
 __device__ __forceinline__ void exp_pack_tile(uint32_t (&sv)[4][32], float c_lo, float b_lo, float c_hi,
                                               float b_hi, bool poly, float& sum_lo, float& sum_hi) {
   uint64_t acc_lo = 0, acc_hi = 0;  // packed partial sums (0.0f, 0.0f)
@@ -104,23 +105,26 @@ __device__ __forceinline__ void exp_pack_tile(uint32_t (&sv)[4][32], float c_lo,
     for (int i = 0; i < 32; i += 2) {
       const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), cc2, bb2);
       uint64_t p;
-      if (kPolyEvery > 0 && poly && ((i >> 1) % kPolyEvery) == kPolyEvery - 1) {
+      if (kPolyEvery > 0 && poly && ((i >> 1) % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
         p = exp2_poly2(x);
       } else {
         p = f2_pack(ex2_approx(f2_lo(x)), ex2_approx(f2_hi(x)));
       }
       const uint32_t packed = kF16 ? pack_f16x2(f2_lo(p), f2_hi(p)) : pack_bf16x2(f2_lo(p), f2_hi(p));
       sv[c & 2][(c & 1) * 16 + (i >> 1)] = packed;
-      // The row sum adds the *rounded* P the MMA multiplies V by, so that
-      // O = sum(P V) / sum(P) uses one set of weights.  With the lazy max a
-      // dominant key's P lies in (1, 2^8] and is inexact in bf16; summing
-      // the rounded value cancels that rounding in the quotient.
-      uint64_t pr;
-      if (kF16) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&packed));
-        pr = f2_pack(f.x, f.y);
-      } else {
-        pr = f2_pack(__uint_as_float(packed << 16), __uint_as_float(packed & 0xFFFF0000u));
+      // With kRoundedSum the row sum adds the *rounded* P the MMA multiplies
+      // V by, so that O = sum(P V) / sum(P) uses one set of weights.  With
+      // the lazy max a dominant key's P lies in (1, 2^8] and is inexact in
+      // bf16 (2^-9); summing the rounded value cancels that rounding in the
+      // quotient.  fp16 P rounds 8x finer, where the fp32 sum is kept.
+      uint64_t pr = p;
+      if (kRoundedSum) {
+        if (kF16) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&packed));
+          pr = f2_pack(f.x, f.y);
+        } else {
+          pr = f2_pack(__uint_as_float(packed << 16), __uint_as_float(packed & 0xFFFF0000u));
+        }
       }
       acc = f2_add(acc, pr);
     }
