@@ -98,6 +98,34 @@ __device__ __forceinline__ uint4 norm_rope_row(const uint4& raw, const float (&w
   return pack8(y);
 }
 
+// As norm_rope_row, also folding max |y| of the unrounded fp32 results into
+// `amax` (rounding to bf16 is monotonic, so rounding the final maximum gives
+// the maximum of the rounded values).
+__device__ __forceinline__ uint4 norm_rope_row_amax(const uint4& raw, const float (&w)[8], const float (&c)[4],
+                                                    const float (&s)[4], float eps, float& amax) {
+  float x[8];
+  unpack8(raw, x);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+  ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+  const float r = rsqrtf(ss * (1.0f / kHeadDim) + eps);
+  float y[8];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const float a0 = x[2 * m] * r * w[2 * m];
+    const float a1 = x[2 * m + 1] * r * w[2 * m + 1];
+    y[2 * m] = fmaf(a0, c[m], -a1 * s[m]);
+    y[2 * m + 1] = fmaf(a0, s[m], a1 * c[m]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[i]));
+  return pack8(y);
+}
+
 __device__ __forceinline__ void load_weights(const float* w, int l16, float (&out)[8]) {
   if (w == nullptr) {
 #pragma unroll
@@ -169,14 +197,17 @@ __global__ void __launch_bounds__(kBf16Warps * 32) prologue_bf16_kernel(const __
 }
 
 // ------------------------------------------------------------- FP8 mode ----
-// One CTA per (64-token block, group of 4 heads, batch); 16 warps, each
-// owning 4 tokens; a half-warp owns one head of a token.  Processed rows
-// stay in registers (bf16-rounded) while the block absmax is reduced in
-// shared memory, then are quantised and stored as E4M3.
-constexpr int kFp8Warps = 16;
-constexpr int kFp8TokPerWarp = kQuantBlock / kFp8Warps;  // 4
-constexpr int kFp8Heads = 4;
-constexpr int kFp8Pairs = kFp8Heads / 2;                 // head pairs per token
+// Two warps per (batch, head, 64-token block), each owning 32 tokens; a
+// half-warp owns one token row, so each lane holds 16 rows of 8 channels
+// (64 registers of packed bf16) from load to store.  The block absmax needs
+// every processed value of the block before any can be quantised: each warp
+// reduces its 32 tokens, the two partners swap their maxima through shared
+// memory and a 64-thread named barrier, then both quantise from registers.
+// A CTA covers kF8Heads heads; the rotation table (cos, sin) of the block's
+// 64 tokens x 64 channel pairs is built once per CTA in shared memory.
+constexpr int kF8Heads = 4;
+constexpr int kF8Threads = 64 * kF8Heads;
+constexpr int kF8Rows = 16;   // rows per lane (32 tokens / 2 half-warps)
 
 __device__ __forceinline__ float absmax8(const uint4& u) {
   // |bf16| as float: clear the sign bit of each half and compare as floats.
@@ -210,9 +241,9 @@ __device__ __forceinline__ uint2 quant8(const uint4& u, float inv) {
   return make_uint2(out[0], out[1]);
 }
 
-__global__ void __launch_bounds__(kFp8Warps * 32) prologue_fp8_kernel(const __grid_constant__ PrologueArgs a) {
-  __shared__ unsigned int s_amax[3][kFp8Heads];
-  __shared__ float s_inv[3][kFp8Heads];
+__global__ void __launch_bounds__(kF8Threads, 2) prologue_fp8_kernel(const __grid_constant__ PrologueArgs a) {
+  __shared__ __align__(16) float2 s_rot[kQuantBlock][64];  // [token][axis * 32 + pair] = (cos, sin)
+  __shared__ float s_amax[kF8Heads][2];                     // [head in CTA][token half]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -220,90 +251,84 @@ __global__ void __launch_bounds__(kFp8Warps * 32) prologue_fp8_kernel(const __gr
   const int l16 = lane & 15;
   const int axis = l16 >> 3;
   const int pair0 = (l16 & 7) * 4;
+  const int hl = warp >> 1;            // head within the CTA
+  const int th = warp & 1;             // token half of the block: tokens [32 th, 32 th + 32)
   const int blk = blockIdx.x;
-  const int hg = blockIdx.y * kFp8Heads;
   const int b = blockIdx.z;
+  const int h = blockIdx.y * kF8Heads + hl;
+  const int t0 = blk * kQuantBlock;
   const int nblk = (a.N + kQuantBlock - 1) / kQuantBlock;
 
-  if (threadIdx.x < 3 * kFp8Heads) s_amax[threadIdx.x / kFp8Heads][threadIdx.x % kFp8Heads] = 0u;
-
-  float c[kFp8TokPerWarp][4], s[kFp8TokPerWarp][4];
+  // Lane's rows: tokens t0 + 32 th + 2 i + half, i = 0..15; uint4 index of
+  // row i is base + i * row_step.
+  const size_t row_step = static_cast<size_t>(2) * a.H * 16;
+  const size_t base = ((static_cast<size_t>(b) * a.N + t0 + 32 * th + half) * a.H + h) * 16 + l16;
+  const int tok0 = 32 * th + half;
+  const int bar_id = 1 + hl;
+  uint4 rows[kF8Rows];
+  auto load_rows = [&](const void* src) {
+    const uint4* in = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-  for (int k = 0; k < kFp8TokPerWarp; ++k) {
-    const int t = blk * kQuantBlock + warp * kFp8TokPerWarp + k;
+    for (int i = 0; i < kF8Rows; ++i)
+      rows[i] = (h < a.H && t0 + tok0 + 2 * i < a.N) ? __ldcs(in + base + i * row_step) : make_uint4(0, 0, 0, 0);
+  };
+  load_rows(a.q);  // in flight while the rotation table is built
+
+  constexpr double kTwoPi = 6.283185307179586476925286766559;
+  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
+  for (int e = threadIdx.x; e < kQuantBlock * 64; e += kF8Threads) {
+    const int tok = e >> 6, pr = e & 63;
     int row = 0, col = 0;
-    if (t < a.N) token_pos(a, t, row, col);
-    lane_rotations(a, axis == 0 ? row : col, pair0, c[k], s[k]);
+    if (t0 + tok < a.N) token_pos(a, t0 + tok, row, col);
+    const double phi = static_cast<double>(pr < 32 ? row : col) * a.omega[pr & 31];
+    const double rr = phi - rint(phi * kInvTwoPi) * kTwoPi;
+    float sn, cs;
+    sincosf(static_cast<float>(rr), &sn, &cs);
+    s_rot[tok][pr] = make_float2(cs, sn);
   }
   __syncthreads();
-
-  const void* ins[3] = {a.q, a.k, a.v};
-  void* outs[3] = {a.q_out, a.k_out, a.v_out};
-  float* scales[3] = {a.q_scale, a.k_scale, a.v_scale};
-  const float* wts[2] = {a.q_w, a.k_w};
+  if (h >= a.H) return;  // both warps of a head leave together; no CTA barrier follows
 
 #pragma unroll 1
   for (int ti = 0; ti < 3; ++ti) {
-    const uint4* in = reinterpret_cast<const uint4*>(ins[ti]);
-    uint4 rows[kFp8TokPerWarp][kFp8Pairs];
-#pragma unroll
-    for (int k = 0; k < kFp8TokPerWarp; ++k) {
-      const int t = blk * kQuantBlock + warp * kFp8TokPerWarp + k;
-#pragma unroll
-      for (int j = 0; j < kFp8Pairs; ++j) {
-        const int h = hg + 2 * j + half;
-        if (t < a.N && h < a.H) {
-          const size_t idx = ((static_cast<size_t>(b) * a.N + t) * a.H + h) * 16 + l16;
-          rows[k][j] = __ldcs(in + idx);
-        } else {
-          rows[k][j] = make_uint4(0, 0, 0, 0);
-        }
-      }
-    }
+    if (ti > 0) load_rows(ti == 1 ? a.k : a.v);
+    float amax = 0.f;
     if (ti < 2) {
       float w[8];
-      load_weights(wts[ti], l16, w);
+      load_weights(ti == 0 ? a.q_w : a.k_w, l16, w);
 #pragma unroll
-      for (int k = 0; k < kFp8TokPerWarp; ++k)
-#pragma unroll
-        for (int j = 0; j < kFp8Pairs; ++j) rows[k][j] = norm_rope_row(rows[k][j], w, c[k], s[k], a.eps);
-    }
-    // Block absmax per head: lanes of a half-warp, 4 tokens, then the CTA.
-#pragma unroll
-    for (int j = 0; j < kFp8Pairs; ++j) {
-      float m = 0.f;
-#pragma unroll
-      for (int k = 0; k < kFp8TokPerWarp; ++k) m = fmaxf(m, absmax8(rows[k][j]));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-      if (l16 == 0) atomicMax(&s_amax[ti][2 * j + half], __float_as_uint(m));
-    }
-    __syncthreads();
-    if (threadIdx.x < kFp8Heads) {
-      const int h = hg + threadIdx.x;
-      const float amax = __uint_as_float(s_amax[ti][threadIdx.x]);
-      const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
-      s_inv[ti][threadIdx.x] = inv;
-      if (h < a.H) {
-        scales[ti][(static_cast<size_t>(b) * a.H + h) * nblk + blk] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      for (int i = 0; i < kF8Rows; ++i) {
+        const int tok = tok0 + 2 * i;
+        const float4 r0 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0]);
+        const float4 r1 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0 + 2]);
+        const float c[4] = {r0.x, r0.z, r1.x, r1.z};
+        const float sn[4] = {r0.y, r0.w, r1.y, r1.w};
+        const bool valid = t0 + tok < a.N;
+        float am = 0.f;
+        const uint4 y = norm_rope_row_amax(rows[i], w, c, sn, a.eps, am);
+        rows[i] = valid ? y : make_uint4(0, 0, 0, 0);
+        amax = valid ? fmaxf(amax, am) : amax;
       }
-    }
-    __syncthreads();
-    uint2* out = reinterpret_cast<uint2*>(outs[ti]);
+      amax = __bfloat162float(__float2bfloat16_rn(amax));
+    } else {
 #pragma unroll
-    for (int k = 0; k < kFp8TokPerWarp; ++k) {
-      const int t = blk * kQuantBlock + warp * kFp8TokPerWarp + k;
-#pragma unroll
-      for (int j = 0; j < kFp8Pairs; ++j) {
-        const int h = hg + 2 * j + half;
-        if (t < a.N && h < a.H) {
-          const size_t idx = ((static_cast<size_t>(b) * a.N + t) * a.H + h) * 16 + l16;
-          __stcs(out + idx, quant8(rows[k][j], s_inv[ti][2 * j + half]));
-        }
-      }
+      for (int i = 0; i < kF8Rows; ++i) amax = fmaxf(amax, absmax8(rows[i]));
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (lane == 0) s_amax[hl][th] = amax;
+    named_bar_sync(bar_id, 64);
+    amax = fmaxf(amax, s_amax[hl][th ^ 1]);
+    named_bar_sync(bar_id, 64);  // both read before either rewrites s_amax for the next tensor
+    const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+    if (th == 0 && lane == 0) {
+      float* sc = ti == 0 ? a.q_scale : (ti == 1 ? a.k_scale : a.v_scale);
+      sc[(static_cast<size_t>(b) * a.H + h) * nblk + blk] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    }
+    uint2* out = reinterpret_cast<uint2*>(ti == 0 ? a.q_out : (ti == 1 ? a.k_out : a.v_out));
+#pragma unroll
+    for (int i = 0; i < kF8Rows; ++i)
+      if (t0 + tok0 + 2 * i < a.N) __stcs(out + base + i * row_step, quant8(rows[i], inv));
   }
 }
 
@@ -317,8 +342,8 @@ cudaError_t launch_prologue_bf16(const PrologueArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_prologue_fp8(const PrologueArgs& a, cudaStream_t s) {
-  dim3 grid((a.N + kQuantBlock - 1) / kQuantBlock, (a.H + kFp8Heads - 1) / kFp8Heads, a.B);
-  prologue_fp8_kernel<<<grid, kFp8Warps * 32, 0, s>>>(a);
+  dim3 grid((a.N + kQuantBlock - 1) / kQuantBlock, (a.H + kF8Heads - 1) / kF8Heads, a.B);
+  prologue_fp8_kernel<<<grid, kF8Threads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
