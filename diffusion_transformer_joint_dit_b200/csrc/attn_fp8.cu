@@ -349,7 +349,8 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint32_t sv[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sv[c]);
-      tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);  // ties the loaded registers to the wait
       const int nvalid = N - j * kBN;
       if (nvalid < kBN) {
 #pragma unroll
@@ -388,7 +389,7 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int c = 0; c < 4; ++c) {
           uint32_t ov[32];
           tmem_ld32(o_addr + c * 32, ov);
-          tmem_ld_wait();
+          tmem_ld_wait(ov);
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
           tmem_st32(o_addr + c * 32, ov);
@@ -407,7 +408,7 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int c = 0; c < 4; ++c) {
         uint32_t ov[32];
         tmem_ld32(o_addr + c * 32, ov);
-        tmem_ld_wait();
+        tmem_ld_wait(ov);
         if (row < N) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
