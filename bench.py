@@ -40,7 +40,7 @@ WORKLOAD = "t2i_2048"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_bf16_t2i_2048.json")
-KERNEL_SOURCES = ["attn_bf16.cu", "sm100_ptx.cuh"]
+KERNEL_SOURCES = ["attn_bf16.cu", "sm100_ptx.cuh", "softmax_sm100.cuh", "jattn_internal.h"]
 
 
 def parse_args():
