@@ -39,7 +39,7 @@ UNIT = "TFLOP/s"
 WORKLOAD = "t2i_2048"
 L2_BYTES = 126 * 2 ** 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_bf16_t2i_2048.json")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_bf16_traffic_t2i_2048.md")
 KERNEL_SOURCES = ["attn_bf16.cu", "sm100_ptx.cuh", "softmax_sm100.cuh", "jattn_internal.h"]
 
 
@@ -91,15 +91,23 @@ def kernel_source_sha() -> str:
 
 def profiled_traffic():
     """DRAM bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel source; else None."""
+    was taken on the current kernel source; else None.  The summary is a
+    Markdown file whose key lines read `- key: value`."""
     try:
         with open(PROFILE_SUMMARY) as f:
-            d = json.load(f)
-    except (OSError, ValueError):
+            kv = {}
+            for line in f:
+                if line.startswith("- ") and ": " in line:
+                    key, val = line[2:].split(": ", 1)
+                    kv[key.strip()] = val.strip().strip("`")
+    except OSError:
         return None
-    if d.get("source_sha256") != kernel_source_sha():
+    if kv.get("source_sha256") != kernel_source_sha():
         return None
-    return d.get("dram_bytes_per_launch")
+    try:
+        return int(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 class ClockSampler:
