@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "jattn.h"
@@ -103,6 +104,37 @@ cudaError_t make_act_map(CUtensorMap* map, const void* ptr, int B, int N, int H,
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t make_rows_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int box_heads, int box_tokens) {
+  EncodeTiledFn fn = encoder();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t row = static_cast<cuuint64_t>(kHeadDim) * 2;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {row, row * H, row * H * N};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(kHeadDim), static_cast<cuuint32_t>(box_heads),
+                       static_cast<cuuint32_t>(box_tokens), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int device_sm_count() {
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cached[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDev) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDev) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 cudaError_t set_smem_attr(const void* func, int bytes) {
   constexpr int kMaxDev = 64;
   constexpr int kMaxFuncs = 8;
@@ -186,6 +218,7 @@ int jattn_prologue(const void* q, const void* k, const void* v, void* q_out, voi
   a.ref_w = p->ref_w > 0 ? p->ref_w : 1;
   a.ref_row_offset = p->ref_row_offset;
   a.eps = p->eps;
+  a.timeout_ns = kDefaultTimeoutNs;
   for (int i = 0; i < 32; ++i) a.omega[i] = std::pow(static_cast<double>(p->rope_theta), -2.0 * i / 64.0);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   return map_err(mode == JATTN_PROLOGUE_BF16 ? launch_prologue_bf16(a, s) : launch_prologue_fp8(a, s));

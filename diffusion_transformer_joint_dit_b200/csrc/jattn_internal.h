@@ -28,6 +28,7 @@ struct PrologueArgs {
   int B, H, N;
   int n_txt, n_img, img_w, ref_w, ref_row_offset;
   float eps;
+  uint64_t timeout_ns;  // bound of each barrier wait (FP8 mode)
   // RoPE frequencies of the 32 channel pairs of one axis half,
   // omega_i = theta^(-2i/64), in double so that angles are exact enough.
   double omega[32];
@@ -60,6 +61,15 @@ cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t s);
 // zero fill out of bounds.  Encoded through cuTensorMapEncodeTiled, looked
 // up via the runtime's driver entry point (no link-time libcuda dependency).
 cudaError_t make_act_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int elem_bytes);
+
+// 4-D tensor map over a token-major bf16 [B, N, H, d=128] tensor for the
+// prologue: box (128 channels, `box_heads` heads, `box_tokens` tokens, 1),
+// no swizzle (rows land densely, 256 B each, token-major then head), zero
+// fill out of bounds.
+cudaError_t make_rows_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int box_heads, int box_tokens);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
 
 // Raise a kernel's dynamic shared-memory limit on the current device (once
 // per device and kernel).

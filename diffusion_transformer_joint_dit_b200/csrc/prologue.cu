@@ -197,17 +197,28 @@ __global__ void __launch_bounds__(kBf16Warps * 32) prologue_bf16_kernel(const __
 }
 
 // ------------------------------------------------------------- FP8 mode ----
-// Two warps per (batch, head, 64-token block), each owning 32 tokens; a
-// half-warp owns one token row, so each lane holds 16 rows of 8 channels
-// (64 registers of packed bf16) from load to store.  The block absmax needs
-// every processed value of the block before any can be quantised: each warp
-// reduces its 32 tokens, the two partners swap their maxima through shared
-// memory and a 64-thread named barrier, then both quantise from registers.
-// A CTA covers kF8Heads heads; the rotation table (cos, sin) of the block's
-// 64 tokens x 64 channel pairs is built once per CTA in shared memory.
-constexpr int kF8Heads = 4;
-constexpr int kF8Threads = 64 * kF8Heads;
-constexpr int kF8Rows = 16;   // rows per lane (32 tokens / 2 half-warps)
+// Persistent kernel.  CTA c processes a contiguous run of work items
+// (64-token block, batch, pair of heads), block-major, so the rotation
+// table of a block (cos, sin of its 64 tokens x 64 channel pairs, 32 KB of
+// shared memory) is built once and reused for every head pair of the block.
+// An item's Q, K and V rows (64 tokens x 2 heads x 256 B = 32 KB each) come
+// in by TMA into one of two shared-memory buffers; the next item's rows
+// land while this one is processed, so HBM stays busy.
+// Warp w handles head w / 8 of the pair and tokens [8 (w mod 8), +8), a
+// half-warp per row: each lane keeps 4 rows of 8 channels in registers
+// from normalisation to quantisation (16 warps per SM hide the latency of
+// the shuffles and conversions).  The block absmax needs every processed
+// value of the block: each warp reduces its 8 tokens, the eight warps of a
+// head meet through shared memory and a 256-thread named barrier, then all
+// quantise from registers.
+constexpr int kF8Pair = 2;                                       // heads per item
+constexpr int kF8WarpsPerHead = 8;
+constexpr int kF8Threads = kF8Pair * kF8WarpsPerHead * 32;       // 512
+constexpr int kF8Rows = kQuantBlock / (2 * kF8WarpsPerHead);     // 4 rows per lane
+constexpr int kF8TileBytes = kQuantBlock * kF8Pair * kHeadDim * 2;  // 32 KB
+constexpr int kF8SmemRot = 0;                                    // float2 [64][64]
+constexpr int kF8SmemBuf = kQuantBlock * 64 * 8;                 // 32 KB
+constexpr int kF8SmemBytes = kF8SmemBuf + 2 * 3 * kF8TileBytes + 1024;  // + alignment slack
 
 __device__ __forceinline__ float absmax8(const uint4& u) {
   // |bf16| as float: clear the sign bit of each half and compare as floats.
@@ -241,9 +252,15 @@ __device__ __forceinline__ uint2 quant8(const uint4& u, float inv) {
   return make_uint2(out[0], out[1]);
 }
 
-__global__ void __launch_bounds__(kF8Threads, 2) prologue_fp8_kernel(const __grid_constant__ PrologueArgs a) {
-  __shared__ __align__(16) float2 s_rot[kQuantBlock][64];  // [token][axis * 32 + pair] = (cos, sin)
-  __shared__ float s_amax[kF8Heads][2];                     // [head in CTA][token half]
+__global__ void __launch_bounds__(kF8Threads, 1)
+prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, int n_items) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float2 (*s_rot)[64] = reinterpret_cast<float2 (*)[64]>(smem + kF8SmemRot);  // [token][axis * 32 + pair]
+  __shared__ uint64_t s_full[2][3];            // [buffer][Q, K, V] rows landed
+  __shared__ float s_amax[kF8Pair][kF8WarpsPerHead];  // [head of the pair][warp of the head]
+  __shared__ int s_abort;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -251,84 +268,136 @@ __global__ void __launch_bounds__(kF8Threads, 2) prologue_fp8_kernel(const __gri
   const int l16 = lane & 15;
   const int axis = l16 >> 3;
   const int pair0 = (l16 & 7) * 4;
-  const int hl = warp >> 1;            // head within the CTA
-  const int th = warp & 1;             // token half of the block: tokens [32 th, 32 th + 32)
-  const int blk = blockIdx.x;
-  const int b = blockIdx.z;
-  const int h = blockIdx.y * kF8Heads + hl;
-  const int t0 = blk * kQuantBlock;
+  const int hl = warp / kF8WarpsPerHead;       // head of the pair
+  const int tq = warp % kF8WarpsPerHead;       // token group of the block
+  const int tok0 = 2 * kF8Rows * tq + half;    // lane's rows: tokens tok0 + 2 i
+  const int bar_id = 1 + hl;                   // the warps of head hl
   const int nblk = (a.N + kQuantBlock - 1) / kQuantBlock;
+  const int n_pairs = (a.H + kF8Pair - 1) / kF8Pair;
+  const int begin = static_cast<int>(static_cast<long long>(blockIdx.x) * n_items / gridDim.x);
+  const int end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * n_items / gridDim.x);
+  const CUtensorMap* maps[3] = {&tm_q, &tm_k, &tm_v};
 
-  // Lane's rows: tokens t0 + 32 th + 2 i + half, i = 0..15; uint4 index of
-  // row i is base + i * row_step.
-  const size_t row_step = static_cast<size_t>(2) * a.H * 16;
-  const size_t base = ((static_cast<size_t>(b) * a.N + t0 + 32 * th + half) * a.H + h) * 16 + l16;
-  const int tok0 = 32 * th + half;
-  const int bar_id = 1 + hl;
-  uint4 rows[kF8Rows];
-  auto load_rows = [&](const void* src) {
-    const uint4* in = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-    for (int i = 0; i < kF8Rows; ++i)
-      rows[i] = (h < a.H && t0 + tok0 + 2 * i < a.N) ? __ldcs(in + base + i * row_step) : make_uint4(0, 0, 0, 0);
+  auto coords = [&](int item, int& blk, int& b, int& hp) {
+    hp = item % n_pairs;
+    const int rest = item / n_pairs;
+    b = rest % a.B;
+    blk = rest / a.B;
   };
-  load_rows(a.q);  // in flight while the rotation table is built
+  auto tile = [&](int buf, int x) { return smem + kF8SmemBuf + (buf * 3 + x) * kF8TileBytes; };
+  // Thread 0: TMA of item `item`'s Q, K, V rows into buffer `buf`.
+  auto issue = [&](int item, int buf) {
+    int blk, b, hp;
+    coords(item, blk, b, hp);
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      mbar_arrive_expect_tx(&s_full[buf][x], kF8TileBytes);
+      tma_load_4d(tile(buf, x), maps[x], &s_full[buf][x], 0, hp * kF8Pair, blk * kQuantBlock, b);
+    }
+  };
+
+  int issued_end = begin;  // thread 0: one past the last item whose copies were issued
+  if (threadIdx.x == 0) {
+    for (int u = 0; u < 2; ++u)
+      for (int x = 0; x < 3; ++x) mbar_init(&s_full[u][x], 1);
+    s_abort = 0;
+    fence_barrier_init();
+    if (begin < end) {
+      for (int x = 0; x < 3; ++x) prefetch_tensormap(maps[x]);
+      issue(begin, 0);
+      issued_end = begin + 1;
+    }
+  }
+  __syncthreads();
 
   constexpr double kTwoPi = 6.283185307179586476925286766559;
   constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
-  for (int e = threadIdx.x; e < kQuantBlock * 64; e += kF8Threads) {
-    const int tok = e >> 6, pr = e & 63;
-    int row = 0, col = 0;
-    if (t0 + tok < a.N) token_pos(a, t0 + tok, row, col);
-    const double phi = static_cast<double>(pr < 32 ? row : col) * a.omega[pr & 31];
-    const double rr = phi - rint(phi * kInvTwoPi) * kTwoPi;
-    float sn, cs;
-    sincosf(static_cast<float>(rr), &sn, &cs);
-    s_rot[tok][pr] = make_float2(cs, sn);
-  }
-  __syncthreads();
-  if (h >= a.H) return;  // both warps of a head leave together; no CTA barrier follows
+  int cur_blk = -1;
+  for (int item = begin; item < end; ++item) {
+    const int i = item - begin;
+    const int buf = i & 1;
+    // Buffer buf ^ 1 was released by the barrier that ended the previous item.
+    if (threadIdx.x == 0 && item + 1 < end && !s_abort) {
+      issue(item + 1, buf ^ 1);
+      issued_end = item + 2;
+    }
+    int blk, b, hp;
+    coords(item, blk, b, hp);
+    const int t0 = blk * kQuantBlock;
+    const int h = hp * kF8Pair + hl;
+    if (blk != cur_blk) {  // same for the whole CTA
+      for (int e = threadIdx.x; e < kQuantBlock * 64; e += kF8Threads) {
+        const int tok = e >> 6, pr = e & 63;
+        int row = 0, col = 0;
+        if (t0 + tok < a.N) token_pos(a, t0 + tok, row, col);
+        const double phi = static_cast<double>(pr < 32 ? row : col) * a.omega[pr & 31];
+        const double rr = phi - rint(phi * kInvTwoPi) * kTwoPi;
+        float sn, cs;
+        sincosf(static_cast<float>(rr), &sn, &cs);
+        s_rot[tok][pr] = make_float2(cs, sn);
+      }
+      __syncthreads();
+      cur_blk = blk;
+    }
 
 #pragma unroll 1
-  for (int ti = 0; ti < 3; ++ti) {
-    if (ti > 0) load_rows(ti == 1 ? a.k : a.v);
-    float amax = 0.f;
-    if (ti < 2) {
-      float w[8];
-      load_weights(ti == 0 ? a.q_w : a.k_w, l16, w);
+    for (int x = 0; x < 3; ++x) {
+      const bool ok = mbar_wait(&s_full[buf][x], static_cast<uint32_t>(i >> 1) & 1u, &s_abort, a.timeout_ns);
+      const uint4* src = reinterpret_cast<const uint4*>(tile(buf, x));
+      uint4 rows[kF8Rows];
 #pragma unroll
-      for (int i = 0; i < kF8Rows; ++i) {
-        const int tok = tok0 + 2 * i;
-        const float4 r0 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0]);
-        const float4 r1 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0 + 2]);
-        const float c[4] = {r0.x, r0.z, r1.x, r1.z};
-        const float sn[4] = {r0.y, r0.w, r1.y, r1.w};
-        const bool valid = t0 + tok < a.N;
-        float am = 0.f;
-        const uint4 y = norm_rope_row_amax(rows[i], w, c, sn, a.eps, am);
-        rows[i] = valid ? y : make_uint4(0, 0, 0, 0);
-        amax = valid ? fmaxf(amax, am) : amax;
+      for (int r = 0; r < kF8Rows; ++r)
+        rows[r] = ok ? src[((tok0 + 2 * r) * kF8Pair + hl) * 16 + l16] : make_uint4(0, 0, 0, 0);
+      float amax = 0.f;
+      if (x < 2) {
+        float w[8];
+        load_weights(x == 0 ? a.q_w : a.k_w, l16, w);
+#pragma unroll
+        for (int r = 0; r < kF8Rows; ++r) {
+          const int tok = tok0 + 2 * r;
+          const float4 r0 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0]);
+          const float4 r1 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0 + 2]);
+          const float c[4] = {r0.x, r0.z, r1.x, r1.z};
+          const float sn[4] = {r0.y, r0.w, r1.y, r1.w};
+          float am = 0.f;
+          rows[r] = norm_rope_row_amax(rows[r], w, c, sn, a.eps, am);
+          amax = t0 + tok < a.N ? fmaxf(amax, am) : amax;
+        }
+        amax = __bfloat162float(__float2bfloat16_rn(amax));
+      } else {
+#pragma unroll
+        for (int r = 0; r < kF8Rows; ++r) amax = fmaxf(amax, absmax8(rows[r]));
       }
-      amax = __bfloat162float(__float2bfloat16_rn(amax));
-    } else {
 #pragma unroll
-      for (int i = 0; i < kF8Rows; ++i) amax = fmaxf(amax, absmax8(rows[i]));
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (lane == 0) s_amax[hl][tq] = amax;
+      named_bar_sync(bar_id, kF8WarpsPerHead * 32);
+#pragma unroll
+      for (int k = 0; k < kF8WarpsPerHead; ++k) amax = fmaxf(amax, s_amax[hl][k]);
+      named_bar_sync(bar_id, kF8WarpsPerHead * 32);  // all read before s_amax is rewritten
+      if (ok && h < a.H) {
+        const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+        if (tq == 0 && lane == 0) {
+          float* sc = x == 0 ? a.q_scale : (x == 1 ? a.k_scale : a.v_scale);
+          sc[(static_cast<size_t>(b) * a.H + h) * nblk + blk] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        }
+        uint2* out = reinterpret_cast<uint2*>(x == 0 ? a.q_out : (x == 1 ? a.k_out : a.v_out));
+#pragma unroll
+        for (int r = 0; r < kF8Rows; ++r) {
+          const int t = t0 + tok0 + 2 * r;
+          if (t < a.N) __stcs(out + ((static_cast<size_t>(b) * a.N + t) * a.H + h) * 16 + l16, quant8(rows[r], inv));
+        }
+      }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) s_amax[hl][th] = amax;
-    named_bar_sync(bar_id, 64);
-    amax = fmaxf(amax, s_amax[hl][th ^ 1]);
-    named_bar_sync(bar_id, 64);  // both read before either rewrites s_amax for the next tensor
-    const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
-    if (th == 0 && lane == 0) {
-      float* sc = ti == 0 ? a.q_scale : (ti == 1 ? a.k_scale : a.v_scale);
-      sc[(static_cast<size_t>(b) * a.H + h) * nblk + blk] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+    __syncthreads();  // buffer buf and the table are free again
+  }
+  // Drain: the last two issued items' copies have landed before the CTA exits.
+  if (threadIdx.x == 0) {
+    int never = 0;
+    for (int item = (issued_end - 2 > begin ? issued_end - 2 : begin); item < issued_end; ++item) {
+      const int i = item - begin;
+      for (int x = 0; x < 3; ++x) mbar_wait(&s_full[i & 1][x], static_cast<uint32_t>(i >> 1) & 1u, &never, a.timeout_ns);
     }
-    uint2* out = reinterpret_cast<uint2*>(ti == 0 ? a.q_out : (ti == 1 ? a.k_out : a.v_out));
-#pragma unroll
-    for (int i = 0; i < kF8Rows; ++i)
-      if (t0 + tok0 + 2 * i < a.N) __stcs(out + base + i * row_step, quant8(rows[i], inv));
   }
 }
 
@@ -342,8 +411,18 @@ cudaError_t launch_prologue_bf16(const PrologueArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_prologue_fp8(const PrologueArgs& a, cudaStream_t s) {
-  dim3 grid((a.N + kQuantBlock - 1) / kQuantBlock, (a.H + kF8Heads - 1) / kF8Heads, a.B);
-  prologue_fp8_kernel<<<grid, kF8Threads, 0, s>>>(a);
+  CUtensorMap tq, tk, tv;
+  cudaError_t e;
+  if ((e = make_rows_map(&tq, a.q, a.B, a.N, a.H, kF8Pair, kQuantBlock)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&tk, a.k, a.B, a.N, a.H, kF8Pair, kQuantBlock)) != cudaSuccess) return e;
+  if ((e = make_rows_map(&tv, a.v, a.B, a.N, a.H, kF8Pair, kQuantBlock)) != cudaSuccess) return e;
+  if ((e = set_smem_attr(reinterpret_cast<const void*>(prologue_fp8_kernel), kF8SmemBytes)) != cudaSuccess) return e;
+  const long long n_items = static_cast<long long>((a.N + kQuantBlock - 1) / kQuantBlock) * a.B *
+                            ((a.H + kF8Pair - 1) / kF8Pair);
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int grid = static_cast<int>(n_items < sms ? n_items : sms);
+  prologue_fp8_kernel<<<grid, kF8Threads, kF8SmemBytes, s>>>(a, tq, tk, tv, static_cast<int>(n_items));
   return cudaGetLastError();
 }
 
