@@ -18,6 +18,7 @@
 
 #include "jattn_internal.h"
 #include "sm100_ptx.cuh"
+#include "softmax_sm100.cuh"
 
 namespace jattn {
 
@@ -100,29 +101,35 @@ __device__ __forceinline__ uint4 norm_rope_row(const uint4& raw, const float (&w
 
 // As norm_rope_row, also folding max |y| of the unrounded fp32 results into
 // `amax` (rounding to bf16 is monotonic, so rounding the final maximum gives
-// the maximum of the rounded values).
+// the maximum of the rounded values).  Sum of squares and the x * r * w
+// products use packed f32x2 arithmetic.
 __device__ __forceinline__ uint4 norm_rope_row_amax(const uint4& raw, const float (&w)[8], const float (&c)[4],
                                                     const float (&s)[4], float eps, float& amax) {
   float x[8];
   unpack8(raw, x);
-  float ss = 0.f;
+  uint64_t x2[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+  for (int m = 0; m < 4; ++m) x2[m] = f2_pack(x[2 * m], x[2 * m + 1]);
+  uint64_t s2 = f2_mul(x2[0], x2[0]);
+#pragma unroll
+  for (int m = 1; m < 4; ++m) s2 = f2_fma(x2[m], x2[m], s2);
+  float ss = f2_lo(s2) + f2_hi(s2);
   ss += __shfl_xor_sync(0xffffffffu, ss, 1);
   ss += __shfl_xor_sync(0xffffffffu, ss, 2);
   ss += __shfl_xor_sync(0xffffffffu, ss, 4);
   ss += __shfl_xor_sync(0xffffffffu, ss, 8);
   const float r = rsqrtf(ss * (1.0f / kHeadDim) + eps);
+  const uint64_t r2 = f2_pack(r, r);
   float y[8];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    const float a0 = x[2 * m] * r * w[2 * m];
-    const float a1 = x[2 * m + 1] * r * w[2 * m + 1];
+    const uint64_t a2 = f2_mul(f2_mul(x2[m], r2), f2_pack(w[2 * m], w[2 * m + 1]));
+    const float a0 = f2_lo(a2), a1 = f2_hi(a2);
     y[2 * m] = fmaf(a0, c[m], -a1 * s[m]);
     y[2 * m + 1] = fmaf(a0, s[m], a1 * c[m]);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[i]));
+  for (int m = 0; m < 4; ++m) amax = fmax3(amax, fabsf(y[2 * m]), fabsf(y[2 * m + 1]));
   return pack8(y);
 }
 
@@ -220,30 +227,30 @@ constexpr int kF8SmemRot = 0;                                    // float2 [64][
 constexpr int kF8SmemBuf = kQuantBlock * 64 * 8;                 // 32 KB
 constexpr int kF8SmemBytes = kF8SmemBuf + 2 * 3 * kF8TileBytes + 1024;  // + alignment slack
 
-__device__ __forceinline__ float absmax8(const uint4& u) {
-  // |bf16| as float: clear the sign bit of each half and compare as floats.
+// max |x| over 8 bf16 as packed 16-bit integers: with the sign bits cleared,
+// bf16 magnitudes order like unsigned integers (inf and NaN excepted, which
+// finite inputs do not produce).  Returns the two 16-bit lane maxima.
+__device__ __forceinline__ uint32_t absmax8_u16x2(const uint4& u, uint32_t m) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-  float m = 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    m = fmaxf(m, __uint_as_float((w[i] << 16) & 0x7FFFFFFFu));
-    m = fmaxf(m, __uint_as_float(w[i] & 0x7FFF0000u));
-  }
+  for (int i = 0; i < 4; ++i) asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(w[i] & 0x7FFF7FFFu));
   return m;
 }
 
 __device__ __forceinline__ uint2 quant8(const uint4& u, float inv) {
   float x[8];
   unpack8(u, x);
+  const uint64_t inv2 = f2_pack(inv, inv);
   uint32_t out[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
     uint32_t word = 0;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
+      const uint64_t p2 = f2_mul(f2_pack(x[4 * i + 2 * j], x[4 * i + 2 * j + 1]), inv2);  // correctly rounded
       float2 f;
-      f.x = __fmul_rn(x[4 * i + 2 * j], inv);
-      f.y = __fmul_rn(x[4 * i + 2 * j + 1], inv);
+      f.x = f2_lo(p2);
+      f.y = f2_hi(p2);
       const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
       word |= static_cast<uint32_t>(p) << (16 * j);
     }
@@ -365,8 +372,10 @@ prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constan
         }
         amax = __bfloat162float(__float2bfloat16_rn(amax));
       } else {
+        uint32_t m2 = 0;
 #pragma unroll
-        for (int r = 0; r < kF8Rows; ++r) amax = fmaxf(amax, absmax8(rows[r]));
+        for (int r = 0; r < kF8Rows; ++r) m2 = absmax8_u16x2(rows[r], m2);
+        amax = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
