@@ -106,6 +106,7 @@ __device__ __forceinline__ void exp_pack_tile(uint32_t (&sv)[4][32], float c_lo,
     const float bb = c < 2 ? b_lo : b_hi;
     const uint64_t cc2 = f2_pack(cc, cc), bb2 = f2_pack(bb, bb);
     uint64_t acc = 0;
+    float acc_a = 0.f, acc_b = 0.f;  // bf16 rounded-sum path: even / odd keys
 #pragma unroll
     for (int i = 0; i < 32; i += 2) {
       const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), cc2, bb2);
@@ -121,18 +122,24 @@ __device__ __forceinline__ void exp_pack_tile(uint32_t (&sv)[4][32], float c_lo,
       // V by, so that O = sum(P V) / sum(P) uses one set of weights.  With
       // the lazy max a dominant key's P lies in (1, 2^8] and is inexact in
       // bf16 (2^-9); summing the rounded value cancels that rounding in the
-      // quotient.  fp16 P rounds 8x finer, where the fp32 sum is kept.
-      uint64_t pr = p;
-      if (kRoundedSum) {
-        if (kF16) {
+      // quotient.  bf16 halves are added straight into fp32 with the
+      // mixed-precision add; fp16 P rounds 8x finer, where the fp32 sum is
+      // kept.
+      if (kRoundedSum && !kF16) {
+        asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+            "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+            : "+f"(acc_a), "+f"(acc_b)
+            : "r"(packed));
+      } else {
+        uint64_t pr = p;
+        if (kRoundedSum) {
           const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&packed));
           pr = f2_pack(f.x, f.y);
-        } else {
-          pr = f2_pack(__uint_as_float(packed << 16), __uint_as_float(packed & 0xFFFF0000u));
         }
+        acc = f2_add(acc, pr);
       }
-      acc = f2_add(acc, pr);
     }
+    if (kRoundedSum && !kF16) acc = f2_pack(acc_a, acc_b);
     if (c < 2) acc_lo = f2_add(acc_lo, acc); else acc_hi = f2_add(acc_hi, acc);
   }
   sum_lo = f2_lo(acc_lo) + f2_hi(acc_lo);
