@@ -54,6 +54,9 @@ def parse_args():
                     help="CPU oracle baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-path timing object")
+    ap.add_argument("--sp", action="store_true",
+                    help="Ulysses sequence parallelism over all ranks (strong scaling of one problem) "
+                         "instead of one independent problem per rank")
     return ap.parse_args()
 
 
@@ -479,6 +482,75 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return 0
 
 
+def run_sp(args, rank: int, world: int, local_rank: int):
+    """One problem split over all ranks by Ulysses sequence parallelism: each
+    rank holds its sequence shard of Q, K, V in HBM; a step is the exchange
+    to head shards, the prologue and BF16 attention on H / P heads, and the
+    exchange back.  Total work is fixed as ranks are added (strong scaling)."""
+    from diffusion_transformer_joint_dit_b200 import binding as J
+    from diffusion_transformer_joint_dit_b200 import ulysses as U
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29531")
+    torch.distributed.init_process_group("nccl", rank=rank, world_size=world,
+                                         timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        w = I.WORKLOADS[args.workload]
+        if w.path != "bf16" or w.H % world != 0:
+            raise SystemExit("--sp needs a BF16 workload whose heads split over the ranks")
+        q, k, v = I.make_qkv(w, seed=0)
+        s0, s1 = U.shard_bounds(w.N, world, rank)
+        qd, kd, vd = (t[:, s0:s1].contiguous().to(dev) for t in (q, k, v))
+        prologue, attn = U.jattn_bf16_ops(w.n_txt, w.n_img, w.n_ref, w.softmax_scale, w.img_h, w.img_w,
+                                          w.ref_h, w.ref_w, w.ref_row_offset)
+
+        def step():
+            return U.ulysses_attention(qd, kd, vd, n_total=w.N, attn=attn, prologue=prologue)
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize(dev)
+        if J.jattn_device_status() != J.JATTN_OK:
+            raise RuntimeError("device error word set during warm-up")
+        K = args.steps
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks = ClockSampler(local_rank)
+        torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        clocks.start()
+        e0.record()
+        for _ in range(K):
+            step()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        clk = clocks.stop()
+        torch.distributed.barrier()
+        if J.jattn_device_status() != J.JATTN_OK:
+            raise RuntimeError("device error word set during the timed region")
+        ms = max_over_ranks([e0.elapsed_time(e1) / K], dev)[0]
+        if rank == 0:
+            value = w.flops / (ms * 1e-3) / 1e12
+            line = {
+                "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+                "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded N(0,1) bf16 Q, K, V)",
+                "config": workload_config(w, {
+                    "path": "bf16", "parallelism": f"ulysses sp{world} (all-to-all over NCCL)",
+                    "step": "all-to-all to head shards + jattn_prologue + jattn_fwd_bf16 on H/P heads + "
+                            "all-to-all back",
+                    "l2": "inputs larger than L2"}),
+                "gpu_launches": 2 * K,
+                "clocks": clk,
+            }
+            print(json.dumps(line), flush=True)
+    finally:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -488,6 +560,8 @@ def main():
         raise SystemExit("--gpus N > 1 runs under torchrun (one process per GPU)")
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.sp:
+        return run_sp(args, rank, world, local_rank)
     return run_ours(args, rank, world, local_rank)
 
 
