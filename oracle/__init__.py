@@ -42,7 +42,9 @@ from .jattn_oracle import (  # noqa: F401
     e4m3_encode,
     joint_attention,
     prologue,
+    qkv_fused,
     rmsnorm,
     rope_2d,
+    rope_table,
     token_positions,
 )

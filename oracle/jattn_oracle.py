@@ -146,6 +146,61 @@ def prologue(q, k, *, n_txt: int, img_h: int, img_w: int,
     return rope_2d(qn, rows, cols, theta), rope_2d(kn, rows, cols, theta)
 
 
+def rope_table(n_txt: int, img_h: int, img_w: int, ref_h: int = 0, ref_w: int = 0,
+               ref_row_offset: int = 0, theta: float = 10000.0) -> np.ndarray:
+    """(cos, sin) of every token's 64 rotation angles, ``[N, 64, 2]`` float64.
+
+    Entry (t, j): angle pos * theta**(-2 (j mod 32) / 64) with pos the row
+    position of token t for j < 32 and its column position for j >= 32 --
+    the angle ``rope_2d`` applies to channel pair (2j, 2j+1) of a 128-wide
+    head.
+    """
+    rows, cols = token_positions(n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset)
+    n = len(rows)
+    out = np.empty((n, 64, 2), dtype=np.float64)
+    for j in range(64):
+        pos = (rows if j < 32 else cols).astype(np.float64)
+        phi = pos * theta ** (-2.0 * (j % 32) / 64.0)
+        out[:, j, 0] = np.cos(phi)
+        out[:, j, 1] = np.sin(phi)
+    return out
+
+
+def qkv_fused(x, w_txt, w_img, *, n_txt: int, img_h: int, img_w: int, H: int,
+              ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0,
+              theta: float = 10000.0, eps: float = 1e-6,
+              q_norm_w=(None, None), k_norm_w=(None, None)):
+    """QKV projection with the prologue in its epilogue, in float64.
+
+    The tutorial's "GEMM kernel optimization" section fuses query/key
+    normalisation and RoPE into the QKV projection; its "FLUX 3 inference"
+    section has the text and image streams processed separately until the
+    joint attention.  Reading: each stream s has its own projection
+    ``W_s`` (``[3 H d, C]``, rows = Q heads, K heads, V heads) and its own
+    Q/K norm weights; reference-image tokens use the image stream's.
+    ``x`` is ``[B, N, C]``.  Returns unrounded float64 ``Q', K', V``
+    ``[B, N, H, d]``: Q' = RoPE(RMSNorm(x W_s,q^T) * q_norm_w[s]), K' likewise,
+    V = x W_s,v^T.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    B, N, C = x.shape
+    d = 128
+    y = np.empty((B, N, 3 * H * d), dtype=np.float64)
+    y[:, :n_txt] = x[:, :n_txt] @ np.asarray(w_txt, dtype=np.float64).T if n_txt > 0 else 0.0
+    if N > n_txt:
+        y[:, n_txt:] = x[:, n_txt:] @ np.asarray(w_img, dtype=np.float64).T
+    q = y[..., :H * d].reshape(B, N, H, d)
+    k = y[..., H * d:2 * H * d].reshape(B, N, H, d)
+    v = y[..., 2 * H * d:].reshape(B, N, H, d)
+    qn = np.empty_like(q)
+    kn = np.empty_like(k)
+    for s, sl in ((0, slice(0, n_txt)), (1, slice(n_txt, N))):
+        qn[:, sl] = rmsnorm(q[:, sl], q_norm_w[s], eps)
+        kn[:, sl] = rmsnorm(k[:, sl], k_norm_w[s], eps)
+    rows, cols = token_positions(n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset)
+    return rope_2d(qn, rows, cols, theta), rope_2d(kn, rows, cols, theta), v
+
+
 # ---------------------------------------------------------------------------
 # E4M3 block quantisation (FP8 path)
 # ---------------------------------------------------------------------------

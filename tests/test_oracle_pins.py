@@ -342,3 +342,89 @@ def test_inputs_are_seeded_and_shaped():
         assert t in rows
     m = I.outlier_rows(I.WORKLOADS["t2i_2048"])
     assert m.sum() == round(0.01 * m.size)
+
+
+# ---------------------------------------------------------------------------
+# RoPE table and the fused QKV projection (NEXT-2)
+# ---------------------------------------------------------------------------
+
+def test_rope_table_closed_form_entries():
+    t = O.rope_table(n_txt=3, img_h=4, img_w=5, ref_h=2, ref_w=2, ref_row_offset=4)
+    assert t.shape == (3 + 20 + 4, 64, 2)
+    np.testing.assert_allclose(t[..., 0] ** 2 + t[..., 1] ** 2, 1.0, atol=1e-15)
+    np.testing.assert_array_equal(t[:3], np.broadcast_to([1.0, 0.0], (3, 64, 2)))   # text at (0, 0)
+    tok = 3 + 2 * 5 + 3                          # image token at (row 2, col 3)
+    assert t[tok, 0].tolist() == [math.cos(2.0), math.sin(2.0)]          # pair 0: pos radians
+    assert t[tok, 32].tolist() == [math.cos(3.0), math.sin(3.0)]
+    phi = 2.0 * math.pow(10000.0, -1.0 / 32.0)                         # pair 1 of the row half
+    np.testing.assert_allclose(t[tok, 1], [math.cos(phi), math.sin(phi)], rtol=0, atol=1e-15)
+    ref = 3 + 20 + 3                              # reference token (row 4 + 1, col 1)
+    assert t[ref, 0].tolist() == [math.cos(5.0), math.sin(5.0)]
+    assert t[ref, 32].tolist() == [math.cos(1.0), math.sin(1.0)]
+
+
+def test_rope_table_is_the_rotation_rope_2d_applies():
+    rows, cols = O.token_positions(2, 3, 4)
+    t = O.rope_table(2, 3, 4)
+    e = np.zeros((1, len(rows), 1, 128))
+    e[..., 0::2] = 1.0                            # unit first element of every pair
+    r = O.rope_2d(e, rows, cols)[0, :, 0]
+    np.testing.assert_allclose(r[:, 0::2], t[..., 0], atol=1e-15)
+    np.testing.assert_allclose(r[:, 1::2], t[..., 1], atol=1e-15)
+
+
+def _qkv_case(C=256, H=2, n_txt=3, img_h=2, img_w=3, seed=5):
+    rng = np.random.default_rng(seed)
+    n = n_txt + img_h * img_w
+    x = rng.standard_normal((2, n, C))
+    w_txt = rng.standard_normal((3 * H * 128, C)) / np.sqrt(C)
+    w_img = rng.standard_normal((3 * H * 128, C)) / np.sqrt(C)
+    return x, w_txt, w_img, dict(n_txt=n_txt, img_h=img_h, img_w=img_w, H=H)
+
+
+def test_qkv_fused_identity_weights_reduce_to_prologue():
+    H, n_txt = 2, 3
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((1, n_txt + 6, H * 128))
+    eye = np.eye(H * 128)
+    w = np.concatenate([eye, eye, eye])           # Q = K = V = x
+    q, k, v = O.qkv_fused(x, w, w, n_txt=n_txt, img_h=2, img_w=3, H=H)
+    xh = x.reshape(1, n_txt + 6, H, 128)
+    qp, kp = O.prologue(xh, xh, n_txt=n_txt, img_h=2, img_w=3)
+    np.testing.assert_array_equal(v, xh)
+    np.testing.assert_allclose(q, qp, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(k, kp, rtol=0, atol=1e-14)
+
+
+def test_qkv_fused_streams_use_their_own_weights():
+    x, w_txt, w_img, kw = _qkv_case()
+    q0, k0, v0 = O.qkv_fused(x, w_txt, w_img, **kw)
+    q1, k1, v1 = O.qkv_fused(x, w_txt, 2.0 * w_img + 1.0, **kw)        # image weights only
+    n = kw["n_txt"]
+    for a, b in ((q0, q1), (k0, k1), (v0, v1)):
+        np.testing.assert_array_equal(a[:, :n], b[:, :n])
+        assert not np.allclose(a[:, n:], b[:, n:])
+    q2, _, v2 = O.qkv_fused(x, 3.0 * w_txt, w_img, **kw)                 # text weights only
+    np.testing.assert_array_equal(q2[:, n:], q0[:, n:])
+    np.testing.assert_allclose(v2[:, :n], 3.0 * v0[:, :n], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(q2[:, :n], q0[:, :n], rtol=0, atol=1e-12)   # RMSNorm removes the scale
+
+
+def test_qkv_fused_value_brute_force_and_norm_weights():
+    x, w_txt, w_img, kw = _qkv_case(C=64, H=2)
+    H = kw["H"]
+    q, k, v = O.qkv_fused(x, w_txt, w_img, **kw)
+    b, t, h, c = 1, 5, 1, 17                      # an image token
+    f = 2 * H * 128 + h * 128 + c
+    want = sum(float(x[b, t, i]) * float(w_img[f, i]) for i in range(64))
+    assert abs(v[b, t, h, c] - want) < 1e-12
+    wq = np.linspace(0.5, 1.5, 128)
+    q2, _, _ = O.qkv_fused(x, w_txt, w_img, q_norm_w=(None, wq), **kw)
+    n = kw["n_txt"]
+    np.testing.assert_array_equal(q2[:, :n], q[:, :n])                    # text tokens untouched
+    # RoPE mixes pairs, so compare the pair norms: weights scale channel-wise
+    # before rotation; with equal weights within a pair the norm scales by it.
+    wq_pairs = np.repeat(np.linspace(0.5, 1.5, 64), 2)
+    q3, _, _ = O.qkv_fused(x, w_txt, w_img, q_norm_w=(None, wq_pairs), **kw)
+    pn = lambda a: np.sqrt(a[..., 0::2] ** 2 + a[..., 1::2] ** 2)
+    np.testing.assert_allclose(pn(q3[:, n:]), pn(q[:, n:]) * wq_pairs[0::2], rtol=1e-12)
