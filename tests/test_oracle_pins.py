@@ -404,10 +404,11 @@ def test_qkv_fused_streams_use_their_own_weights():
     for a, b in ((q0, q1), (k0, k1), (v0, v1)):
         np.testing.assert_array_equal(a[:, :n], b[:, :n])
         assert not np.allclose(a[:, n:], b[:, n:])
-    q2, _, v2 = O.qkv_fused(x, 3.0 * w_txt, w_img, **kw)                 # text weights only
-    np.testing.assert_array_equal(q2[:, n:], q0[:, n:])
+    q2, _, v2 = O.qkv_fused(x, 3.0 * w_txt, w_img, eps=0.0, **kw)       # text weights only
+    q0e, _, _ = O.qkv_fused(x, w_txt, w_img, eps=0.0, **kw)
+    np.testing.assert_array_equal(q2[:, n:], q0e[:, n:])
     np.testing.assert_allclose(v2[:, :n], 3.0 * v0[:, :n], rtol=1e-12, atol=1e-13)
-    np.testing.assert_allclose(q2[:, :n], q0[:, :n], rtol=0, atol=1e-12)   # RMSNorm removes the scale
+    np.testing.assert_allclose(q2[:, :n], q0e[:, :n], rtol=0, atol=1e-12)  # RMSNorm (eps 0) removes the scale
 
 
 def test_qkv_fused_value_brute_force_and_norm_weights():
