@@ -27,9 +27,9 @@ JATTN_PROLOGUE_BF16 = 0
 JATTN_PROLOGUE_FP8 = 1
 JATTN_FP8_BLOCK = 64
 
-EXPORTED = ("jattn_prologue", "jattn_fwd_bf16", "jattn_fwd_fp8", "jattn_status_string",
-            "jattn_device_status", "jattn_selftest_wait_timeout", "jattn_selftest_exp2_poly",
-            "jattn_last_cuda_error")
+EXPORTED = ("jattn_prologue", "jattn_fwd_bf16", "jattn_fwd_fp8", "jattn_rope_table", "jattn_qkv_fused",
+            "jattn_status_string", "jattn_device_status", "jattn_selftest_wait_timeout",
+            "jattn_selftest_exp2_poly", "jattn_last_cuda_error")
 
 
 class JattnError(RuntimeError):
@@ -48,6 +48,15 @@ class jattn_prologue_params(ctypes.Structure):
         ("ref_row_offset", ctypes.c_int),
         ("rope_theta", ctypes.c_float), ("eps", ctypes.c_float),
         ("q_norm_w", ctypes.c_void_p), ("k_norm_w", ctypes.c_void_p),
+    ]
+
+
+class jattn_qkv_weights(ctypes.Structure):
+    _fields_ = [
+        ("w_qkv", ctypes.c_void_p * 2),
+        ("q_norm_w", ctypes.c_void_p * 2),
+        ("k_norm_w", ctypes.c_void_p * 2),
+        ("eps", ctypes.c_float),
     ]
 
 
@@ -72,6 +81,11 @@ def load_library():
     lib.jattn_fwd_bf16.restype = _I
     lib.jattn_fwd_fp8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]
     lib.jattn_fwd_fp8.restype = _I
+    lib.jattn_rope_table.argtypes = [_P, _I, _I, _I, ctypes.POINTER(jattn_prologue_params), _P]
+    lib.jattn_rope_table.restype = _I
+    lib.jattn_qkv_fused.argtypes = [_P, ctypes.POINTER(jattn_qkv_weights), _P, _P, _P, _P,
+                                    _I, _I, _I, _I, _I, _I, _I, _P]
+    lib.jattn_qkv_fused.restype = _I
     lib.jattn_status_string.argtypes = [_I]
     lib.jattn_status_string.restype = ctypes.c_char_p
     lib.jattn_device_status.argtypes = [_P]
@@ -151,6 +165,35 @@ def jattn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B: int, H: int,
                                       softmax_scale, _stream(stream))
     if check:
         _check("jattn_fwd_fp8", st)
+    return st
+
+
+def make_qkv_weights(w_txt, w_img, q_norm_w=(None, None), k_norm_w=(None, None), eps: float = 1e-6):
+    """jattn_qkv_weights from per-stream tensors (text, image + reference)."""
+    wt = jattn_qkv_weights()
+    wt.w_qkv[0], wt.w_qkv[1] = _ptr(w_txt), _ptr(w_img)
+    wt.q_norm_w[0], wt.q_norm_w[1] = _ptr(q_norm_w[0]), _ptr(q_norm_w[1])
+    wt.k_norm_w[0], wt.k_norm_w[1] = _ptr(k_norm_w[0]), _ptr(k_norm_w[1])
+    wt.eps = eps
+    return wt
+
+
+def jattn_rope_table(table, N_txt: int, N_img: int, N_ref: int, params: jattn_prologue_params, stream=None, *,
+                     check: bool = True) -> int:
+    st = load_library().jattn_rope_table(_ptr(table), N_txt, N_img, N_ref,
+                                         ctypes.byref(params) if params is not None else None, _stream(stream))
+    if check:
+        _check("jattn_rope_table", st)
+    return st
+
+
+def jattn_qkv_fused(x, weights: jattn_qkv_weights, rope, q, k, v, B: int, H: int, N_txt: int, N_img: int,
+                    N_ref: int, d: int, C: int, stream=None, *, check: bool = True) -> int:
+    st = load_library().jattn_qkv_fused(_ptr(x), ctypes.byref(weights) if weights is not None else None,
+                                        _ptr(rope), _ptr(q), _ptr(k), _ptr(v), B, H, N_txt, N_img, N_ref, d, C,
+                                        _stream(stream))
+    if check:
+        _check("jattn_qkv_fused", st)
     return st
 
 

@@ -14,6 +14,7 @@
 
 #include "attn_bf16.cu"
 #include "attn_fp8.cu"
+#include "qkv_gemm.cu"
 #include "prologue.cu"
 
 namespace jattn {
@@ -116,6 +117,19 @@ cudaError_t make_rows_map(CUtensorMap* map, const void* ptr, int B, int N, int H
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_kmajor_map(CUtensorMap* map, const void* ptr, long long rows, int cols, int box_rows) {
+  EncodeTiledFn fn = encoder();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -266,6 +280,61 @@ int jattn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q
   cudaError_t e = launch_attn_fp8(pr, static_cast<cudaStream_t>(cuda_stream));
   if (e == cudaErrorNotSupported) return JATTN_ERR_UNSUPPORTED;
   return map_err(e);
+}
+
+int jattn_rope_table(float* table, int N_txt, int N_img, int N_ref, const jattn_prologue_params* p,
+                     void* cuda_stream) {
+  int st = check_common(1, 1, N_txt, N_img, N_ref, kHeadDim);
+  if (st != JATTN_OK) return st;
+  if (table == nullptr || p == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(table)) return JATTN_ERR_MISALIGNED;
+  if (p->img_h < 0 || p->img_w < 0 || p->ref_h < 0 || p->ref_w < 0 || p->ref_row_offset < 0)
+    return JATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(p->img_h) * p->img_w != N_img || static_cast<long long>(p->ref_h) * p->ref_w != N_ref)
+    return JATTN_ERR_INVALID_ARG;
+  if (!(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta)) return JATTN_ERR_INVALID_ARG;
+  PrologueArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = 1; a.H = 1; a.N = N_txt + N_img + N_ref;
+  a.n_txt = N_txt; a.n_img = N_img;
+  a.img_w = p->img_w > 0 ? p->img_w : 1;
+  a.ref_w = p->ref_w > 0 ? p->ref_w : 1;
+  a.ref_row_offset = p->ref_row_offset;
+  for (int i = 0; i < 32; ++i) a.omega[i] = std::pow(static_cast<double>(p->rope_theta), -2.0 * i / 64.0);
+  return map_err(launch_rope_table(a, table, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+int jattn_qkv_fused(const void* x, const jattn_qkv_weights* w, const float* rope, void* q, void* k, void* v,
+                    int B, int H, int N_txt, int N_img, int N_ref, int d, int C, void* cuda_stream) {
+  int st = check_common(B, H, N_txt, N_img, N_ref, d);
+  if (st != JATTN_OK) return st;
+  if (H % 2 != 0) return JATTN_ERR_UNSUPPORTED;
+  if (C < 64 || C > 16384 || C % 64 != 0) return JATTN_ERR_UNSUPPORTED;
+  if (x == nullptr || w == nullptr || rope == nullptr || q == nullptr || k == nullptr || v == nullptr)
+    return JATTN_ERR_INVALID_ARG;
+  if ((N_txt > 0 && w->w_qkv[0] == nullptr) || (N_img + N_ref > 0 && w->w_qkv[1] == nullptr))
+    return JATTN_ERR_INVALID_ARG;
+  if (!(w->eps >= 0.f) || !std::isfinite(w->eps)) return JATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * (N_txt + N_img + N_ref) * C * 2 >= (1ll << 40)) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(rope) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(w->w_qkv[0]) || !aligned16(w->w_qkv[1]))
+    return JATTN_ERR_MISALIGNED;
+  for (int s = 0; s < 2; ++s)
+    if (!aligned16(w->q_norm_w[s]) || !aligned16(w->k_norm_w[s])) return JATTN_ERR_MISALIGNED;
+  QkvProblem pr;
+  std::memset(&pr, 0, sizeof(pr));
+  pr.x = x;
+  for (int s = 0; s < 2; ++s) {
+    pr.w[s] = w->w_qkv[s];
+    pr.qw[s] = w->q_norm_w[s];
+    pr.kw[s] = w->k_norm_w[s];
+  }
+  pr.rope = rope;
+  pr.q = q; pr.k = k; pr.v = v;
+  pr.B = B; pr.H = H; pr.N = N_txt + N_img + N_ref; pr.n_txt = N_txt; pr.C = C;
+  pr.eps = w->eps;
+  pr.timeout_ns = kDefaultTimeoutNs;
+  return map_err(launch_qkv_fused(pr, static_cast<cudaStream_t>(cuda_stream)));
 }
 
 const char* jattn_last_cuda_error(void) { return cudaGetErrorName(t_last_cuda_error); }

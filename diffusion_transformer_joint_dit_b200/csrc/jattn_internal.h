@@ -51,6 +51,24 @@ struct AttnProblem {
   uint64_t timeout_ns;
 };
 
+// Fused QKV projection (qkv_gemm.cu).
+struct QkvProblem {
+  const void* x;        // bf16 [B, N, C]
+  const void* w[2];     // bf16 [3 H d, C] per stream (text, image + reference)
+  const float* qw[2];   // [d] per stream, nullable
+  const float* kw[2];
+  const float* rope;    // [N, 64, 2]
+  void* q;
+  void* k;
+  void* v;
+  int B, H, N, n_txt, C;
+  float eps;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_qkv_fused(const QkvProblem& q, cudaStream_t s);
+cudaError_t launch_rope_table(const PrologueArgs& a, float* table, cudaStream_t s);
+
 cudaError_t launch_attn_bf16(const AttnProblem& p, cudaStream_t s);
 cudaError_t launch_attn_fp8(const AttnProblem& p, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t s);
@@ -67,6 +85,11 @@ cudaError_t make_act_map(CUtensorMap* map, const void* ptr, int B, int N, int H,
 // no swizzle (rows land densely, 256 B each, token-major then head), zero
 // fill out of bounds.
 cudaError_t make_rows_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int box_heads, int box_tokens);
+
+// 2-D tensor map over a row-major bf16 [rows, cols] matrix read K-major:
+// box (64 columns = 128 B, box_rows rows), 128-byte swizzle, zero fill out
+// of bounds.
+cudaError_t make_kmajor_map(CUtensorMap* map, const void* ptr, long long rows, int cols, int box_rows);
 
 // Number of SMs of the current device (cached per device).
 int device_sm_count();

@@ -156,3 +156,23 @@ def random_e4m3_codes(shape, seed: int = 0) -> np.ndarray:
     c = rng.integers(0, 256, size=shape, dtype=np.int64)
     c = np.where((c & 0x7F) == 0x7F, c ^ 0x01, c)
     return c.astype(np.uint8)
+
+
+def make_qkv_projection_inputs(w: Workload, C: int, seed: int = 0):
+    """Inputs of the fused QKV projection as bf16 / fp32 CPU tensors.
+
+    Draw order with ``numpy.random.default_rng(seed)``: activations
+    x ``[B, N, C]`` standard normal; then per stream (text, image) the
+    projection ``[3 H d, C]`` with entries N(0, 1/C), so projected features
+    are about unit size; then per stream the Q and K norm weights
+    ``[d]`` uniform in [0.5, 1.5).
+    Returns ``x, (w_txt, w_img), (qn_txt, qn_img), (kn_txt, kn_img)``.
+    """
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((w.B, w.N, C), dtype=np.float32)
+    ws = [rng.standard_normal((3 * w.H * w.d, C), dtype=np.float32) / np.float32(np.sqrt(C)) for _ in range(2)]
+    qn, kn = [], []
+    for _ in range(2):
+        qn.append(torch.from_numpy(rng.uniform(0.5, 1.5, w.d).astype(np.float32)))
+        kn.append(torch.from_numpy(rng.uniform(0.5, 1.5, w.d).astype(np.float32)))
+    return _to_bf16(x), (_to_bf16(ws[0]), _to_bf16(ws[1])), tuple(qn), tuple(kn)

@@ -10,7 +10,8 @@
  * query/key normalisation and rotary position embedding into the QKV
  * projection epilogue; its "Quantized and sparse attention" section runs the
  * attention itself either in BF16 or with FP8 Q/K and FP8 V.  The three
- * calls below are those steps:
+ * calls below are those steps (jattn_qkv_fused, further down, is the
+ * projection with the prologue fused into its epilogue):
  *
  *   jattn_prologue   per-head RMSNorm of Q and K, 2-D RoPE on the tokens'
  *                    (row, col) latent-grid positions, optionally followed
@@ -163,6 +164,62 @@ JATTN_API int jattn_fwd_fp8(const void* q8, const void* k8, const void* v8,
                   int B, int H, int N_txt, int N_img, int N_ref, int d,
                   float softmax_scale, void* cuda_stream);
 
+/*
+ * jattn_rope_table — the (cos, sin) of every token's 64 RoPE channel pairs,
+ * for jattn_qkv_fused.
+ *
+ * table : fp32 [N, 64, 2] device output; entry (t, j) = (cos phi, sin phi)
+ *         with phi = pos * rope_theta^(-2 (j mod 32) / 64), pos = the row
+ *         position of token t for j < 32, its column position for j >= 32
+ *         (positions as for jattn_prologue; p's norm fields are ignored).
+ * Angles are formed and reduced to [-pi, pi] in double, then evaluated in
+ * float.  N = N_txt + N_img + N_ref >= 1; table 16-byte aligned.
+ */
+JATTN_API int jattn_rope_table(float* table, int N_txt, int N_img, int N_ref,
+                     const jattn_prologue_params* p, void* cuda_stream);
+
+/*
+ * Weights of the fused QKV projection, per token stream.  The tutorial's DiT
+ * processes the text and image streams separately until the joint
+ * attention, so each stream has its own projection and Q/K norm weights;
+ * reference-image tokens use the image stream's (they are latents of the
+ * same kind).  Index 0 = text, 1 = image (and reference).
+ *
+ * w_qkv[s]    : bf16 [3 H d, C] device pointer, row-major: output feature f
+ *               (f < H d: Q head f / d channel f mod d; then K, then V) is
+ *               the dot product of a token's C inputs with row f.
+ * q_norm_w[s], k_norm_w[s] : [d] fp32 device pointers, or NULL for 1.0.
+ * eps         : RMSNorm epsilon (>= 0).
+ */
+typedef struct {
+  const void* w_qkv[2];
+  const float* q_norm_w[2];
+  const float* k_norm_w[2];
+  float eps;
+} jattn_qkv_weights;
+
+/*
+ * jattn_qkv_fused — QKV projection with query/key RMSNorm and 2-D RoPE in
+ * the GEMM epilogue, the fusion the tutorial's "GEMM kernel optimization"
+ * section describes, in BF16 (tcgen05 MMAs, fp32 accumulation).
+ *
+ * x       : bf16 [B, N, C] token activations, the joint sequence
+ *           [text | image | reference] of each batch element.
+ * w       : per-stream weights (see jattn_qkv_weights); w_qkv[0] may be
+ *           NULL when N_txt == 0, w_qkv[1] when N_img + N_ref == 0.
+ * rope    : fp32 [N, 64, 2] from jattn_rope_table.
+ * q, k, v : bf16 [B, N, H, d] outputs.  For token t of stream s:
+ *           Q = RoPE(RMSNorm(x_t W_s,q) * q_norm_w[s]), K likewise with the
+ *           K rows and k_norm_w[s], V = x_t W_s,v; each is rounded to bf16
+ *           once, from the fp32 accumulator (no intermediate rounding).
+ * Sizes: d == 128; H even (two heads per output tile); C a multiple of 64,
+ * 64 <= C <= 16384; N >= 1.  Pointers 16-byte aligned.  The outputs must
+ * not overlap x or the weights.
+ */
+JATTN_API int jattn_qkv_fused(const void* x, const jattn_qkv_weights* w, const float* rope,
+                    void* q, void* k, void* v,
+                    int B, int H, int N_txt, int N_img, int N_ref, int d, int C, void* cuda_stream);
+
 /* Human-readable name of a jattn_status value (static string, never NULL). */
 JATTN_API const char* jattn_status_string(int status);
 
@@ -192,8 +249,9 @@ JATTN_API int jattn_selftest_wait_timeout(long long timeout_ns, void* cuda_strea
 
 /*
  * jattn_selftest_exp2_poly — evaluate, for n floats x (device pointers), the
- * range-reduced polynomial exp2 the attention softmax uses for part of its
- * exponentials, writing y[i] ~ 2^x[i].  Lets tests check its error bound
+ * range-reduced polynomial exp2 the attention softmax can use for a share of
+ * its exponentials (built in, switched off: all-MUFU measured faster),
+ * writing y[i] ~ 2^x[i].  Lets tests check its error bound
  * (relative 7.5e-5 from the degree-3 minimax fit, for x in [-125, 8];
  * smaller x is clamped to -125).
  * n >= 1; x and y 8-byte aligned; asynchronous on cuda_stream.

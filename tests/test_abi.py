@@ -116,6 +116,46 @@ def test_fwd_fp8_rejects_bad_arguments(lib):
     assert call(qs=A + 1) == J.JATTN_ERR_MISALIGNED
 
 
+def qkv(weights="default", **kw):
+    args = dict(x=A, rope=A, q=A, k=A, v=A, B=1, H=2, N_txt=32, N_img=256, N_ref=0, d=128, C=256)
+    args.update(kw)
+    if weights == "default":
+        weights = J.make_qkv_weights(A, A)
+    return J.jattn_qkv_fused(args["x"], weights, args["rope"], args["q"], args["k"], args["v"], args["B"],
+                             args["H"], args["N_txt"], args["N_img"], args["N_ref"], args["d"], args["C"],
+                             stream=0, check=False)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(H=3), J.JATTN_ERR_UNSUPPORTED),                             # two heads per output tile
+    (dict(C=96), J.JATTN_ERR_UNSUPPORTED),                            # not a multiple of 64
+    (dict(C=0), J.JATTN_ERR_UNSUPPORTED),
+    (dict(d=64), J.JATTN_ERR_UNSUPPORTED),
+    (dict(weights=None), J.JATTN_ERR_INVALID_ARG),
+    (dict(weights=J.make_qkv_weights(None, A)), J.JATTN_ERR_INVALID_ARG),   # text tokens, no text weights
+    (dict(weights=J.make_qkv_weights(A, None)), J.JATTN_ERR_INVALID_ARG),   # image tokens, no image weights
+    (dict(weights=J.make_qkv_weights(A, A, eps=-1.0)), J.JATTN_ERR_INVALID_ARG),
+    (dict(weights=J.make_qkv_weights(A, A, q_norm_w=(A + 4, None))), J.JATTN_ERR_MISALIGNED),
+    (dict(rope=None), J.JATTN_ERR_INVALID_ARG),
+    (dict(x=MIS), J.JATTN_ERR_MISALIGNED),
+    (dict(v=MIS), J.JATTN_ERR_MISALIGNED),
+    (dict(N_txt=0, N_img=0), J.JATTN_ERR_INVALID_ARG),
+])
+def test_qkv_fused_rejects_bad_arguments(lib, kw, status):
+    assert qkv(**kw) == status
+
+
+def test_rope_table_rejects_bad_arguments(lib):
+    call = lambda table=A, n_img=256, params="default": J.jattn_rope_table(
+        table, 32, n_img, 0, J.make_prologue_params(16, 16) if params == "default" else params,
+        stream=0, check=False)
+    assert call(table=None) == J.JATTN_ERR_INVALID_ARG
+    assert call(table=MIS) == J.JATTN_ERR_MISALIGNED
+    assert call(params=None) == J.JATTN_ERR_INVALID_ARG
+    assert call(n_img=255) == J.JATTN_ERR_INVALID_ARG
+    assert call(params=J.make_prologue_params(16, 16, rope_theta=-1.0)) == J.JATTN_ERR_INVALID_ARG
+
+
 def test_selftest_rejects_bad_timeout(lib):
     assert J.jattn_selftest_wait_timeout(0, stream=0, check=False) == J.JATTN_ERR_INVALID_ARG
     assert J.jattn_selftest_wait_timeout(2 * 10 ** 9, stream=0, check=False) == J.JATTN_ERR_INVALID_ARG
