@@ -3,23 +3,29 @@
 // fusion the NVIDIA tutorial on FLUX 3 Image Klein describes in its "GEMM
 // kernel optimization" section (there with FP8/NVFP4 weights; here BF16).
 //
-// Design: persistent CTAs, one per SM, each walking output tiles of 128
-// tokens x 256 features (two heads) with a static stride.
-//   warp 0     TMA producer: per 64-channel K step, the x tile (128 x 64,
-//              16 KB) and the stream's W tile (256 x 64, 32 KB) into a
-//              4-stage ring (128-byte swizzle, K-major)
-//   warp 1     TMEM allocator and the single MMA-issuing thread
-//              (tcgen05.mma M=128 N=256 K=16, fp32 accumulation)
-//   warps 2-5  epilogue: TMEM lane quarter = warp mod 4, one token row
-//              per thread
+// Design: persistent clusters of two CTAs (one per SM) sharing
+// tcgen05.mma.cta_group::2 M=256 N=256 K=16: a pair computes an output tile
+// of 256 tokens x 256 features (two heads); CTA r of the pair holds the
+// tile's tokens [128 r, 128 r + 128) as its A operand and features
+// [128 r, 128 r + 128) as its half of B, and receives its 128 token rows
+// of the accumulator in its own TMEM.  Each SM thus takes 32 KB per
+// 64-channel K step from L2 instead of 48 KB (one-SM tiles of the same
+// shape measured L2-bound at about 74% of the tensor peak).
+//   warp 0     TMA producer (both CTAs): its A rows and B half per K step
+//              into a 6-stage ring (128-byte swizzle, K-major); completion
+//              is counted on the leader's barrier
+//   warp 1     TMEM allocator (both CTAs, paired allocation); the leader's
+//              lane 0 issues every MMA of the pair
+//   warps 2-5  epilogue (both CTAs): TMEM lane quarter = warp mod 4, one
+//              token row per thread
 // Two 256-column TMEM accumulators let the epilogue of one tile overlap the
-// main loop of the next.  A tile's 128 rows belong to one (batch, stream):
-// the tile list enumerates each batch element's text rows, then its
-// image + reference rows, in 128-row tiles; rows past the stream's end are
-// computed but not stored.  Because a 256-feature tile holds whole heads,
-// a thread owns all 128 channels of its row's head: the RMSNorm sum of
-// squares is a thread-local loop (first pass over TMEM), the scaling,
-// weights and rotation a second pass, 32 channels at a time.
+// main loop of the next.  A tile's rows belong to one (batch, stream): the
+// tile list enumerates each batch element's text rows, then its image +
+// reference rows, in 256-row tiles; rows past the stream's end are computed
+// but not stored.  Because a tile holds whole heads, a thread owns all 128
+// channels of its row's head: the RMSNorm sum of squares is a thread-local
+// loop (first pass over TMEM), the scaling, weights and rotation a second
+// pass, 32 channels at a time.
 #include "jattn_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -27,26 +33,27 @@ namespace jattn {
 
 namespace qkvgemm {
 
-constexpr int kBM = 128;                       // tokens per tile (= TMEM lanes)
+constexpr int kBM = 128;                       // tokens per CTA (= TMEM lanes); 256 per pair
 constexpr int kBN = 256;                       // output features per tile (two heads)
+constexpr int kBNh = kBN / 2;                  // features per CTA (its half of B)
 constexpr int kBK = 64;                        // input channels per stage (128 B: one swizzle atom)
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kABytes = kBM * kBK * 2;         // 16 KB
-constexpr int kBBytes = kBN * kBK * 2;         // 32 KB
-constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kBBytes = kBNh * kBK * 2;        // 16 KB
+constexpr int kStageBytes = kABytes + kBBytes; // per CTA; the leader's barrier counts both CTAs
 constexpr int kD = 128;
 constexpr int kLoadWarp = 0;
 constexpr int kMmaWarp = 1;
-constexpr int kEpiWarp0 = 2;
 constexpr int kThreads = 6 * 32;
 constexpr uint32_t kTmemCols = 512;            // two accumulators of kBN columns
+constexpr uint16_t kPairMask = 0x3;
 
 struct Ctrl {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t acc_full[2];    // accumulator a holds a finished tile (MMA commit)
-  uint64_t acc_empty[2];   // accumulator a drained by the 128 epilogue threads
-  uint64_t mma_done;
+  uint64_t full[kStages];  // leader: stage s of both CTAs landed
+  uint64_t empty[kStages]; // each CTA: stage s consumed by the pair's MMAs
+  uint64_t acc_full[2];    // each CTA: accumulator a holds a finished tile
+  uint64_t acc_empty[2];   // leader: accumulator a drained by both CTAs' epilogues
+  uint64_t mma_done;       // each CTA: every pair MMA complete
   uint32_t tmem_base;
   int abort;
 };
@@ -62,7 +69,7 @@ struct Params {
   __nv_bfloat16* out[3];    // Q, K, V [B, N, H, d]
   int B, N, H, n_txt;
   int k_steps;              // C / 64
-  int tiles_txt, tiles_img; // 128-row tiles per batch element and stream
+  int tiles_txt, tiles_img; // 256-row tiles per batch element and stream
   int n_tiles_n;            // 3 H d / 256
   int n_tiles;
   float eps;
@@ -82,11 +89,11 @@ __device__ __forceinline__ Tile tile_at(const Params& p, int t) {
   const int r = mt - x.b * per_b;
   if (r < p.tiles_txt) {
     x.stream = 0;
-    x.tok0 = r * kBM;
+    x.tok0 = r * 2 * kBM;
     x.tok_end = p.n_txt;
   } else {
     x.stream = 1;
-    x.tok0 = p.n_txt + (r - p.tiles_txt) * kBM;
+    x.tok0 = p.n_txt + (r - p.tiles_txt) * 2 * kBM;
     x.tok_end = p.N;
   }
   return x;
@@ -106,6 +113,9 @@ qkv_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   volatile int* abort_flag = &ctrl->abort;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();     // 0 = leader
+  const int pair = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -114,18 +124,18 @@ qkv_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ctrl->acc_full[a], 1);
-      mbar_init(&ctrl->acc_empty[a], 4 * 32);
+      mbar_init(&ctrl->acc_empty[a], 2 * 4 * 32);
     }
     mbar_init(&ctrl->mma_done, 1);
     ctrl->abort = 0;
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&ctrl->tmem_base, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&ctrl->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
 
@@ -135,12 +145,14 @@ qkv_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       prefetch_tensormap(&tm_x);
       prefetch_tensormap(&tm_w0);
       prefetch_tensormap(&tm_w1);
+      const uint32_t full0 = mapa_shared(smem_u32(&ctrl->full[0]), 0);  // leader's barriers
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x) {
+      for (int t = pair; t < p.n_tiles && ok; t += n_pairs) {
         const Tile tl = tile_at(p, t);
         const CUtensorMap* wmap = tl.stream == 0 ? &tm_w0 : &tm_w1;
-        const int row0 = tl.b * p.N + tl.tok0;
+        const int row0 = tl.b * p.N + tl.tok0 + kBM * static_cast<int>(rank);
+        const int f0 = tl.nt * kBN + kBNh * static_cast<int>(rank);
         for (int ks = 0; ks < p.k_steps; ++ks, ++it) {
           const int s = it % kStages;
           if (!mbar_wait(&ctrl->empty[s], (static_cast<uint32_t>(it / kStages) & 1u) ^ 1u, abort_flag,
@@ -149,63 +161,70 @@ qkv_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             break;
           }
           uint8_t* st = smem + kSmemRing + s * kStageBytes;
-          mbar_arrive_expect_tx(&ctrl->full[s], kStageBytes);
-          tma_load_2d(st, &tm_x, &ctrl->full[s], ks * kBK, row0);
-          tma_load_2d(st + kABytes, wmap, &ctrl->full[s], ks * kBK, tl.nt * kBN);
+          if (rank == 0) mbar_arrive_expect_tx(&ctrl->full[s], 2 * kStageBytes);
+          tma_load_2d_pair(st, &tm_x, full0 + s * 8, ks * kBK, row0);
+          tma_load_2d_pair(st + kABytes, wmap, full0 + s * 8, ks * kBK, f0);
         }
       }
-      // Drain: every fill issued has landed before the CTA may exit.
-      for (int s = 0; s < kStages && s < it; ++s) {
-        const int last = s + ((it - 1 - s) / kStages) * kStages;
-        drain_wait(&ctrl->full[s], static_cast<uint32_t>(last / kStages) & 1u, p.timeout_ns);
+      // Drain (leader): every fill of both CTAs has landed on its barriers.
+      if (rank == 0) {
+        for (int s = 0; s < kStages && s < it; ++s) {
+          const int last = s + ((it - 1 - s) / kStages) * kStages;
+          drain_wait(&ctrl->full[s], static_cast<uint32_t>(last / kStages) & 1u, p.timeout_ns);
+        }
       }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------- MMA issuer ----
+    // ------------------------------------------------- MMA issuer (leader) ----
     if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc(1, 1, false, kBM, kBN);  // bf16 x bf16, both K-major
-      const uint32_t ring = smem_u32(smem + kSmemRing);
-      int it = 0;
-      bool ok = true;
-      int lt = 0;
-      for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++lt) {
-        const int a = lt & 1;
-        ok = mbar_wait(&ctrl->acc_empty[a], (static_cast<uint32_t>(lt >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t d = tmem + a * kBN;
-        for (int ks = 0; ks < p.k_steps; ++ks, ++it) {
-          const int s = it % kStages;
-          ok = mbar_wait(&ctrl->full[s], static_cast<uint32_t>(it / kStages) & 1u, abort_flag, p.timeout_ns);
+      if (rank == 0) {
+        constexpr uint32_t idesc = make_idesc(1, 1, false, 2 * kBM, kBN);  // M=256 over the pair
+        const uint32_t ring = smem_u32(smem + kSmemRing);
+        int it = 0;
+        bool ok = true;
+        int lt = 0;
+        for (int t = pair; t < p.n_tiles && ok; t += n_pairs, ++lt) {
+          const int a = lt & 1;
+          ok = mbar_wait(&ctrl->acc_empty[a], (static_cast<uint32_t>(lt >> 1) & 1u) ^ 1u, abort_flag,
+                         p.timeout_ns);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sa = ring + s * kStageBytes;
-          const uint32_t sb = sa + kABytes;
+          const uint32_t d = tmem + a * kBN;
+          for (int ks = 0; ks < p.k_steps; ++ks, ++it) {
+            const int s = it % kStages;
+            // TMA-filled stage: its completion is what the barrier reports,
+            // so the MMAs may read it right after the wait.
+            ok = mbar_wait(&ctrl->full[s], static_cast<uint32_t>(it / kStages) & 1u, abort_flag, p.timeout_ns);
+            if (!ok) break;
+            const uint32_t sa = ring + s * kStageBytes;
+            const uint32_t sb = sa + kABytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            mma_f16_ss(d, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024), idesc,
-                       (ks > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              mma_f16_ss_pair(d, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sb + kk * 32, 16, 1024),
+                              idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit_pair(&ctrl->empty[s], kPairMask);
           }
-          mma_commit(&ctrl->empty[s]);
+          if (!ok) break;
+          mma_commit_pair(&ctrl->acc_full[a], kPairMask);
         }
-        if (!ok) break;
-        mma_commit(&ctrl->acc_full[a]);
+        mma_commit_pair(&ctrl->mma_done, kPairMask);
       }
-      // Drain: all issued MMAs complete before TMEM is released.
-      mma_commit(&ctrl->mma_done);
+      // Both CTAs: no TMEM release before every pair MMA has completed.
       drain_wait(&ctrl->mma_done, 0, p.timeout_ns);
     }
     __syncwarp();
   } else {
     // --------------------------------------------------------- epilogue ----
     const int wq = warp & 3;                   // TMEM lane quarter
-    const int r = wq * 32 + lane;              // row within the tile
+    const int r = wq * 32 + lane;              // row within this CTA's half of the tile
     const uint32_t lane_sel = static_cast<uint32_t>(wq * 32) << 16;
     const int HD = p.H * kD;
+    const uint32_t acc_empty0 = mapa_shared(smem_u32(&ctrl->acc_empty[0]), 0);  // leader's barriers
     int lt = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.n_tiles && ok; t += gridDim.x, ++lt) {
+    for (int t = pair; t < p.n_tiles && ok; t += n_pairs, ++lt) {
       const int a = lt & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->acc_full[a], static_cast<uint32_t>(lt >> 1) & 1u, abort_flag,
                                              p.timeout_ns));
@@ -215,7 +234,7 @@ qkv_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       const int f0 = tl.nt * kBN;
       const int part = f0 / HD;                // 0 = Q, 1 = K, 2 = V
       const int h0 = (f0 - part * HD) / kD;
-      const int tok = tl.tok0 + r;
+      const int tok = tl.tok0 + kBM * static_cast<int>(rank) + r;
       const bool store = tok < tl.tok_end;
       const float* nw = part == 0 ? p.qw[tl.stream] : (part == 1 ? p.kw[tl.stream] : nullptr);
       const float* rope = p.rope + static_cast<size_t>(store ? tok : 0) * 128;
@@ -289,15 +308,15 @@ qkv_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         }
       }
       tc_fence_before();
-      mbar_arrive(&ctrl->acc_empty[a]);
+      mbar_arrive_cluster(acc_empty0 + a * 8);
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair may still touch its memory
   if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -311,8 +330,8 @@ cudaError_t launch_qkv_fused(const QkvProblem& q, cudaStream_t s) {
   if ((e = make_kmajor_map(&tx, q.x, rows, q.C, kBM)) != cudaSuccess) return e;
   const void* w0 = q.w[0] != nullptr ? q.w[0] : q.w[1];
   const void* w1 = q.w[1] != nullptr ? q.w[1] : q.w[0];
-  if ((e = make_kmajor_map(&tw0, w0, 3LL * q.H * kD, q.C, kBN)) != cudaSuccess) return e;
-  if ((e = make_kmajor_map(&tw1, w1, 3LL * q.H * kD, q.C, kBN)) != cudaSuccess) return e;
+  if ((e = make_kmajor_map(&tw0, w0, 3LL * q.H * kD, q.C, kBNh)) != cudaSuccess) return e;
+  if ((e = make_kmajor_map(&tw1, w1, 3LL * q.H * kD, q.C, kBNh)) != cudaSuccess) return e;
   if ((e = set_smem_attr(reinterpret_cast<const void*>(qkv_fused_kernel), kSmemBytes)) != cudaSuccess) return e;
   Params p;
   p.rope = q.rope;
@@ -328,8 +347,8 @@ cudaError_t launch_qkv_fused(const QkvProblem& q, cudaStream_t s) {
   p.H = q.H;
   p.n_txt = q.n_txt;
   p.k_steps = q.C / kBK;
-  p.tiles_txt = (q.n_txt + kBM - 1) / kBM;
-  p.tiles_img = (q.N - q.n_txt + kBM - 1) / kBM;
+  p.tiles_txt = (q.n_txt + 2 * kBM - 1) / (2 * kBM);
+  p.tiles_img = (q.N - q.n_txt + 2 * kBM - 1) / (2 * kBM);
   p.n_tiles_n = 3 * q.H * kD / kBN;
   const long long n_tiles = static_cast<long long>(q.B) * (p.tiles_txt + p.tiles_img) * p.n_tiles_n;
   if (n_tiles > 0x7fffffff) return cudaErrorInvalidValue;
@@ -337,9 +356,26 @@ cudaError_t launch_qkv_fused(const QkvProblem& q, cudaStream_t s) {
   p.eps = q.eps;
   p.timeout_ns = q.timeout_ns;
   const int sms = device_sm_count();
-  if (sms <= 0) return cudaErrorInvalidDevice;
-  const int grid = p.n_tiles < sms ? p.n_tiles : sms;
-  qkv_fused_kernel<<<grid, kThreads, kSmemBytes, s>>>(tx, tw0, tw1, p);
+  if (sms < 2) return cudaErrorInvalidDevice;
+  const int pairs = p.n_tiles < sms / 2 ? p.n_tiles : sms / 2;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, qkv_fused_kernel, tx, tw0, tw1, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e;
+  }
   return cudaGetLastError();
 }
 
