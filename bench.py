@@ -54,6 +54,7 @@ def parse_args():
                     help="CPU oracle baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-path timing object")
+    ap.add_argument("--no-qkv", action="store_true", help="skip the fused-QKV-projection timing object")
     ap.add_argument("--sp", action="store_true",
                     help="Ulysses sequence parallelism over all ranks (strong scaling of one problem) "
                          "instead of one independent problem per rank")
@@ -299,6 +300,75 @@ def time_fp8_path(J, dev, stream, rank: int, peaks, peaks_src, steps: int = 10):
     }
 
 
+def time_qkv_fused(J, dev, stream, rank: int, peaks, peaks_src, steps: int = 10):
+    """Fused QKV projection (RMSNorm + RoPE in the GEMM epilogue) on the
+    t2i_2048 shapes: x [B, N, C = H d] -> Q, K, V [B, N, H, d], per-stream
+    weights.  For context it also times the same projection unfused: torch's
+    bf16 matmul (cuBLAS, one per stream) followed by jattn_prologue.
+    Reported beside the headline line, not instead of it."""
+    w = I.WORKLOADS["t2i_2048"]
+    C = w.H * w.d
+    x, (wt, wi), qn, kn = I.make_qkv_projection_inputs(w, C, seed=rank)
+    x, wt, wi = x.to(dev), wt.to(dev), wi.to(dev)
+    qn = tuple(t.to(dev) for t in qn)
+    kn = tuple(t.to(dev) for t in kn)
+    h = stream.cuda_stream
+    rope = torch.empty((w.N, 64, 2), dtype=torch.float32, device=dev)
+    params = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps)
+    J.jattn_rope_table(rope, w.n_txt, w.n_img, w.n_ref, params, h)
+    shape = (w.B, w.N, w.H, w.d)
+    q, k, v = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    wts = J.make_qkv_weights(wt, wi, qn, kn, w.eps)
+    y = torch.empty((w.B, w.N, 3 * C), dtype=torch.bfloat16, device=dev)
+    qu, ku = torch.empty(shape, dtype=torch.bfloat16, device=dev), torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    pparams = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps,
+                                     qn[1], kn[1])
+
+    def fused():
+        J.jattn_qkv_fused(x, wts, rope, q, k, v, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d, C, h)
+
+    def unfused():
+        torch.matmul(x[:, :w.n_txt], wt.T, out=y[:, :w.n_txt])
+        torch.matmul(x[:, w.n_txt:], wi.T, out=y[:, w.n_txt:])
+        yq = y[..., :C].unflatten(-1, (w.H, w.d))
+        yk = y[..., C:2 * C].unflatten(-1, (w.H, w.d))
+        qc, kc = yq.contiguous(), yk.contiguous()
+        J.jattn_prologue(qc, kc, None, qu, ku, None, None, None, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref,
+                         w.d, J.JATTN_PROLOGUE_BF16, pparams, h)
+
+    def timed(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+            torch.cuda.synchronize(dev)
+            for a, b in evs:
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize(dev)
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    ms = timed(fused)
+    if J.jattn_device_status(h) != J.JATTN_OK:
+        raise RuntimeError("device error word set during QKV timing")
+    ms_unfused = timed(unfused)
+    flops = 2.0 * w.B * w.N * C * 3 * C
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {
+        "workload": f"t2i_2048 QKV projection: x [{w.B}, {w.N}, {C}] bf16, per-stream W [{3 * C}, {C}], "
+                    f"Q/K RMSNorm + 2-D RoPE fused",
+        "steps": steps, "ms": ms, "value": achieved, "unit": UNIT,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "peak_source": f"{peaks_src} bf16_tflops",
+                     "flops_per_launch": flops},
+        "unfused_ms": ms_unfused,
+        "unfused_note": "torch bf16 matmul per stream (cuBLAS) + jattn_prologue on Q, K (context, not ours)",
+        "gpu_launches_per_step": 1,
+    }
+
+
 def max_over_ranks(values, device):
     """Element-wise max of per-rank timings over all ranks (identity at N=1)."""
     t = torch.tensor(values, dtype=torch.float64, device=device)
@@ -475,6 +545,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     }
     if not args.no_fp8:
         line["fp8_path"] = time_fp8_path(J, dev, stream, rank, peaks, peaks_src)
+    if not args.no_qkv:
+        line["qkv_fused"] = time_qkv_fused(J, dev, stream, rank, peaks, peaks_src)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k_: v_ for k_, v_ in cpu_baseline(w, q, k, v, args.cpu_seconds).items()
                                 if k_ != "seconds"}
