@@ -43,6 +43,9 @@ from .jattn_oracle import (  # noqa: F401
     joint_attention,
     prologue,
     qkv_fused,
+    repair_count,
+    repair_select,
+    repaired_attention,
     rmsnorm,
     rope_2d,
     rope_table,

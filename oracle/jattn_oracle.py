@@ -334,3 +334,59 @@ __all__ = [
     "rope_2d", "prologue", "e4m3_decode", "e4m3_encode", "block_quantize_e4m3",
     "dequantize_e4m3", "joint_attention",
 ]
+
+
+# ---------------------------------------------------------------------------
+# FP8 attention with a repair budget (VC-Attention style)
+# ---------------------------------------------------------------------------
+
+def repair_count(n: int, rho: float) -> int:
+    """Tokens repaired per (b, h): ceil(rho * N), at most N (0 for rho 0)."""
+    return min(n, int(np.ceil(rho * n - 1e-9))) if rho > 0 else 0
+
+
+def repair_select(k_exact, v_exact, k_deq, v_deq, rho: float):
+    """Key/value tokens with the highest quantisation error, per (b, h).
+
+    The tutorial's "Quantized and sparse attention" section runs
+    VC-Attention FP8 with a repair budget rho = 0.005 that selects the
+    fraction of tokens with the highest quantisation error for residual
+    correction, without defining the error.  Reading: the error of token t
+    of (b, h) is the squared distance between its exact key and value rows
+    (the bf16 K' and V the prologue quantises) and their dequantised E4M3
+    values, summed over the d channels of both:
+
+        e_t = sum_c (K'_tc - Kd_tc)^2 + sum_c (V_tc - Vd_tc)^2,
+
+    and the ``repair_count(N, rho)`` tokens with the largest e_t (ties to the
+    lower token index) are selected.  Returns ``idx int64 [B, H, m]`` (the
+    selected tokens in increasing token order) and the errors ``[B, H, N]``
+    (float64).
+    """
+    ke, ve = np.asarray(k_exact, np.float64), np.asarray(v_exact, np.float64)
+    kd, vd = np.asarray(k_deq, np.float64), np.asarray(v_deq, np.float64)
+    B, N, H, d = ke.shape
+    err = np.transpose(np.sum((ke - kd) ** 2, axis=-1) + np.sum((ve - vd) ** 2, axis=-1), (0, 2, 1))
+    m = repair_count(N, rho)
+    idx = np.empty((B, H, m), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            # Stable sort on -err: equal errors keep increasing token order.
+            idx[b, h] = np.sort(np.argsort(-err[b, h], kind="stable")[:m])
+    return idx, err
+
+
+def repaired_attention(q_deq, k_deq, v_deq, k_exact, v_exact, idx, scale: float):
+    """FP8 attention whose selected keys are repaired: for each (b, h), the
+    tokens in ``idx[b, h]`` attend with their exact K' and V rows, all other
+    keys with the dequantised ones; queries stay dequantised.  Returns
+    ``O [B, N, H, d]`` and ``L [B, H, N]`` (float64), as joint_attention."""
+    k = np.array(k_deq, dtype=np.float64)
+    v = np.array(v_deq, dtype=np.float64)
+    B, N, H, d = k.shape
+    for b in range(B):
+        for h in range(H):
+            t = np.asarray(idx[b, h])
+            k[b, t, h, :] = np.asarray(k_exact, np.float64)[b, t, h, :]
+            v[b, t, h, :] = np.asarray(v_exact, np.float64)[b, t, h, :]
+    return joint_attention(q_deq, k, v, scale)

@@ -429,3 +429,52 @@ def test_qkv_fused_value_brute_force_and_norm_weights():
     q3, _, _ = O.qkv_fused(x, w_txt, w_img, q_norm_w=(None, wq_pairs), **kw)
     pn = lambda a: np.sqrt(a[..., 0::2] ** 2 + a[..., 1::2] ** 2)
     np.testing.assert_allclose(pn(q3[:, n:]), pn(q[:, n:]) * wq_pairs[0::2], rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# FP8 repair budget (NEXT-3)
+# ---------------------------------------------------------------------------
+
+def test_repair_count():
+    assert O.repair_count(16896, 0.005) == 85          # ceil(84.48)
+    assert O.repair_count(200, 0.005) == 1
+    assert O.repair_count(100, 0.0) == 0
+    assert O.repair_count(10, 1.0) == 10 and O.repair_count(10, 2.0) == 10
+    assert O.repair_count(1000, 0.002) == 2            # exact product: no extra token
+
+
+def test_repair_select_hand_case():
+    # 1 batch, 1 head, 6 tokens, d = 2.  Errors: token 0: 1 (K), 1: 4 (V),
+    # 2: 0, 3: 4 (2 from K, 2 from V), 4: 9, 5: 4.
+    ke = np.zeros((1, 6, 1, 2)); kd = np.zeros_like(ke)
+    ve = np.zeros_like(ke); vd = np.zeros_like(ke)
+    kd[0, 0, 0, 0] = 1.0                 # e = 1
+    vd[0, 1, 0, 1] = 2.0                 # e = 4
+    kd[0, 3, 0, :] = 1.0; vd[0, 3, 0, :] = -1.0             # e = 2 + 2 = 4
+    ke[0, 4, 0, 1] = 3.0                 # e = 9
+    ve[0, 5, 0, 0] = -2.0                # e = 4
+    idx, err = O.repair_select(ke, ve, kd, vd, rho=0.5)   # m = 3
+    np.testing.assert_allclose(err[0, 0], [1, 4, 0, 4, 9, 4], rtol=1e-12)
+    # Largest: 4 (9), then the ties at 4 in token order: 1, 3 (5 is left out).
+    assert idx[0, 0].tolist() == [1, 3, 4]
+
+
+def test_repaired_attention_limits():
+    rng = np.random.default_rng(11)
+    shape = (1, 70, 2, 128)
+    ke, ve, qd = (rng.standard_normal(shape) for _ in range(3))
+    kd = ke + 0.05 * rng.standard_normal(shape)
+    vd = ve + 0.05 * rng.standard_normal(shape)
+    none = np.zeros((1, 2, 0), dtype=np.int64)
+    o0, l0 = O.repaired_attention(qd, kd, vd, ke, ve, none, 0.09)
+    r0, rl0 = O.joint_attention(qd, kd, vd, 0.09)
+    np.testing.assert_array_equal(o0, r0)                               # no budget: plain FP8
+    np.testing.assert_array_equal(l0, rl0)
+    allk = np.broadcast_to(np.arange(70), (1, 2, 70))
+    o1, _ = O.repaired_attention(qd, kd, vd, ke, ve, allk, 0.09)
+    r1, _ = O.joint_attention(qd, ke, ve, 0.09)
+    np.testing.assert_allclose(o1, r1, rtol=0, atol=1e-15)             # full budget: exact K, V
+    # A partial budget on the worst tokens moves the result toward exact.
+    idx, _ = O.repair_select(ke, ve, kd, vd, rho=0.3)
+    oh, _ = O.repaired_attention(qd, kd, vd, ke, ve, idx, 0.09)
+    assert np.linalg.norm(oh - r1) < np.linalg.norm(o0 - r1)
