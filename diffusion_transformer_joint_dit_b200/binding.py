@@ -28,6 +28,7 @@ JATTN_PROLOGUE_FP8 = 1
 JATTN_FP8_BLOCK = 64
 
 EXPORTED = ("jattn_prologue", "jattn_fwd_bf16", "jattn_fwd_fp8", "jattn_rope_table", "jattn_qkv_fused",
+            "jattn_fp8_repair_select", "jattn_fp8_repair_apply",
             "jattn_status_string", "jattn_device_status", "jattn_selftest_wait_timeout",
             "jattn_selftest_exp2_poly", "jattn_last_cuda_error")
 
@@ -86,6 +87,12 @@ def load_library():
     lib.jattn_qkv_fused.argtypes = [_P, ctypes.POINTER(jattn_qkv_weights), _P, _P, _P, _P,
                                     _I, _I, _I, _I, _I, _I, _I, _P]
     lib.jattn_qkv_fused.restype = _I
+    lib.jattn_fp8_repair_select.argtypes = [_P, _P, _P, _P, _P, _P, ctypes.POINTER(jattn_prologue_params), _I,
+                                            _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
+    lib.jattn_fp8_repair_select.restype = _I
+    lib.jattn_fp8_repair_apply.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
+                                           _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]
+    lib.jattn_fp8_repair_apply.restype = _I
     lib.jattn_status_string.argtypes = [_I]
     lib.jattn_status_string.restype = ctypes.c_char_p
     lib.jattn_device_status.argtypes = [_P]
@@ -194,6 +201,35 @@ def jattn_qkv_fused(x, weights: jattn_qkv_weights, rope, q, k, v, B: int, H: int
                                         _stream(stream))
     if check:
         _check("jattn_qkv_fused", st)
+    return st
+
+
+def repair_count(n: int, rho: float) -> int:
+    """Tokens repaired per (b, h) for budget rho: ceil(rho * N), at most N."""
+    import math
+    return min(n, math.ceil(rho * n - 1e-9)) if rho > 0 else 0
+
+
+def jattn_fp8_repair_select(k, v, k8, v8, k_scale, v_scale, params: jattn_prologue_params, m: int, err, idx,
+                            k_sel, v_sel, B: int, H: int, N_txt: int, N_img: int, N_ref: int, d: int,
+                            stream=None, *, check: bool = True) -> int:
+    st = load_library().jattn_fp8_repair_select(
+        _ptr(k), _ptr(v), _ptr(k8), _ptr(v8), _ptr(k_scale), _ptr(v_scale),
+        ctypes.byref(params) if params is not None else None, m, _ptr(err), _ptr(idx), _ptr(k_sel), _ptr(v_sel),
+        B, H, N_txt, N_img, N_ref, d, _stream(stream))
+    if check:
+        _check("jattn_fp8_repair_select", st)
+    return st
+
+
+def jattn_fp8_repair_apply(q8, q_scale, k8, v8, k_scale, v_scale, idx, k_sel, v_sel, m: int, o, lse, B: int,
+                           H: int, N_txt: int, N_img: int, N_ref: int, d: int, softmax_scale: float, stream=None,
+                           *, check: bool = True) -> int:
+    st = load_library().jattn_fp8_repair_apply(
+        _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(v8), _ptr(k_scale), _ptr(v_scale), _ptr(idx), _ptr(k_sel),
+        _ptr(v_sel), m, _ptr(o), _ptr(lse), B, H, N_txt, N_img, N_ref, d, softmax_scale, _stream(stream))
+    if check:
+        _check("jattn_fp8_repair_apply", st)
     return st
 
 

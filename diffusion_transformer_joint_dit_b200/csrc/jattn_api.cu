@@ -16,6 +16,7 @@
 #include "attn_fp8.cu"
 #include "qkv_gemm.cu"
 #include "prologue.cu"
+#include "repair.cu"
 
 namespace jattn {
 
@@ -335,6 +336,86 @@ int jattn_qkv_fused(const void* x, const jattn_qkv_weights* w, const float* rope
   pr.eps = w->eps;
   pr.timeout_ns = kDefaultTimeoutNs;
   return map_err(launch_qkv_fused(pr, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+namespace {
+
+// Fills the prologue arguments (positions, RoPE frequencies, norm) shared
+// by jattn_prologue and the repair selection; returns a jattn_status.
+int fill_prologue_args(PrologueArgs& a, const void* q, const void* k, const void* v, int B, int H, int N_txt,
+                       int N_img, int N_ref, const jattn_prologue_params* p) {
+  if (p == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (p->img_h < 0 || p->img_w < 0 || p->ref_h < 0 || p->ref_w < 0 || p->ref_row_offset < 0)
+    return JATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(p->img_h) * p->img_w != N_img || static_cast<long long>(p->ref_h) * p->ref_w != N_ref)
+    return JATTN_ERR_INVALID_ARG;
+  if (!(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta) || !(p->eps >= 0.f) || !std::isfinite(p->eps))
+    return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(p->q_norm_w) || !aligned16(p->k_norm_w)) return JATTN_ERR_MISALIGNED;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k = k; a.v = v;
+  a.q_w = p->q_norm_w; a.k_w = p->k_norm_w;
+  a.B = B; a.H = H; a.N = N_txt + N_img + N_ref;
+  a.n_txt = N_txt; a.n_img = N_img;
+  a.img_w = p->img_w > 0 ? p->img_w : 1;
+  a.ref_w = p->ref_w > 0 ? p->ref_w : 1;
+  a.ref_row_offset = p->ref_row_offset;
+  a.eps = p->eps;
+  a.timeout_ns = kDefaultTimeoutNs;
+  for (int i = 0; i < 32; ++i) a.omega[i] = std::pow(static_cast<double>(p->rope_theta), -2.0 * i / 64.0);
+  return JATTN_OK;
+}
+
+}  // namespace
+
+int jattn_fp8_repair_select(const void* k, const void* v, const void* k8, const void* v8, const float* k_scale,
+                            const float* v_scale, const jattn_prologue_params* p, int m, float* err, int* idx,
+                            void* k_sel, void* v_sel, int B, int H, int N_txt, int N_img, int N_ref, int d,
+                            void* cuda_stream) {
+  int st = check_common(B, H, N_txt, N_img, N_ref, d);
+  if (st != JATTN_OK) return st;
+  const int N = N_txt + N_img + N_ref;
+  if (m < 0 || m > N) return JATTN_ERR_INVALID_ARG;
+  if (k == nullptr || v == nullptr || k8 == nullptr || v8 == nullptr || k_scale == nullptr || v_scale == nullptr ||
+      err == nullptr || (m > 0 && (idx == nullptr || k_sel == nullptr || v_sel == nullptr)))
+    return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k8) || !aligned16(v8) || !aligned16(k_sel) || !aligned16(v_sel) ||
+      ((reinterpret_cast<uintptr_t>(k_scale) | reinterpret_cast<uintptr_t>(v_scale) |
+        reinterpret_cast<uintptr_t>(err) | reinterpret_cast<uintptr_t>(idx)) & 3u))
+    return JATTN_ERR_MISALIGNED;
+  PrologueArgs a;
+  if ((st = fill_prologue_args(a, nullptr, k, v, B, H, N_txt, N_img, N_ref, p)) != JATTN_OK) return st;
+  RepairProblem r;
+  std::memset(&r, 0, sizeof(r));
+  r.k8 = k8; r.v8 = v8; r.k_scale = k_scale; r.v_scale = v_scale;
+  r.err = err; r.idx = idx; r.k_sel = k_sel; r.v_sel = v_sel; r.m = m;
+  return map_err(launch_repair_select(a, r, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+int jattn_fp8_repair_apply(const void* q8, const float* q_scale, const void* k8, const void* v8, const float* k_scale,
+                           const float* v_scale, const int* idx, const void* k_sel, const void* v_sel, int m,
+                           void* o, float* lse, int B, int H, int N_txt, int N_img, int N_ref, int d,
+                           float softmax_scale, void* cuda_stream) {
+  int st = check_common(B, H, N_txt, N_img, N_ref, d);
+  if (st != JATTN_OK) return st;
+  const int N = N_txt + N_img + N_ref;
+  if (m < 0 || m > N) return JATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return JATTN_ERR_INVALID_ARG;
+  if (q8 == nullptr || q_scale == nullptr || k8 == nullptr || v8 == nullptr || k_scale == nullptr ||
+      v_scale == nullptr || o == nullptr || lse == nullptr ||
+      (m > 0 && (idx == nullptr || k_sel == nullptr || v_sel == nullptr)))
+    return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(k_sel) || !aligned16(v_sel) || !aligned16(o) ||
+      ((reinterpret_cast<uintptr_t>(q_scale) | reinterpret_cast<uintptr_t>(k_scale) |
+        reinterpret_cast<uintptr_t>(v_scale) | reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(lse)) &
+       3u))
+    return JATTN_ERR_MISALIGNED;
+  RepairProblem r;
+  std::memset(&r, 0, sizeof(r));
+  r.q8 = q8; r.q_scale = q_scale; r.k8 = k8; r.v8 = v8; r.k_scale = k_scale; r.v_scale = v_scale;
+  r.idx = const_cast<int*>(idx); r.k_sel = const_cast<void*>(k_sel); r.v_sel = const_cast<void*>(v_sel);
+  r.o = o; r.lse = lse; r.m = m;
+  return map_err(launch_repair_apply(r, B, H, N, softmax_scale, static_cast<cudaStream_t>(cuda_stream)));
 }
 
 const char* jattn_last_cuda_error(void) { return cudaGetErrorName(t_last_cuda_error); }

@@ -69,6 +69,26 @@ struct QkvProblem {
 cudaError_t launch_qkv_fused(const QkvProblem& q, cudaStream_t s);
 cudaError_t launch_rope_table(const PrologueArgs& a, float* table, cudaStream_t s);
 
+// FP8 repair budget (repair.cu).
+struct RepairProblem {
+  const void* q8;
+  const float* q_scale;
+  const void* k8;
+  const void* v8;
+  const float* k_scale;
+  const float* v_scale;
+  float* err;         // [B, H, N]
+  int* idx;           // [B, H, m]
+  void* k_sel;        // bf16 [B, H, m, d]
+  void* v_sel;
+  void* o;            // bf16 [B, N, H, d], corrected in place
+  float* lse;         // [B, H, N], corrected in place
+  int m;
+};
+
+cudaError_t launch_repair_select(const PrologueArgs& a, const RepairProblem& r, cudaStream_t s);
+cudaError_t launch_repair_apply(const RepairProblem& r, int B, int H, int N, float softmax_scale, cudaStream_t s);
+
 cudaError_t launch_attn_bf16(const AttnProblem& p, cudaStream_t s);
 cudaError_t launch_attn_fp8(const AttnProblem& p, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t s);

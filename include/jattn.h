@@ -220,6 +220,62 @@ JATTN_API int jattn_qkv_fused(const void* x, const jattn_qkv_weights* w, const f
                     void* q, void* k, void* v,
                     int B, int H, int N_txt, int N_img, int N_ref, int d, int C, void* cuda_stream);
 
+/*
+ * FP8 attention with a repair budget (the tutorial's VC-Attention FP8 runs
+ * with a budget rho = 0.005 that "selects the fraction of tokens with the
+ * highest quantisation error for residual correction"; "Quantized and
+ * sparse attention" section).  Reading implemented, per (batch, head):
+ * the m tokens whose key and value rows lost the most in E4M3,
+ *   e_t = sum_c (K'_tc - Kd_tc)^2 + sum_c (V_tc - Vd_tc)^2
+ * (K' = the bf16 RMSNorm + RoPE of K the prologue quantises, V the bf16
+ * input, Kd / Vd their dequantised codes), are attended with their exact
+ * rows instead of the dequantised ones; queries stay dequantised.  The
+ * tutorial's budget is m = ceil(rho N) (85 at N = 16896).
+ *
+ * Usage: jattn_prologue(mode FP8) -> jattn_fwd_fp8 (with lse) ->
+ * jattn_fp8_repair_select -> jattn_fp8_repair_apply.
+ */
+
+/*
+ * jattn_fp8_repair_select — per-token errors and the selected tokens.
+ *
+ * k, v              : bf16 [B, N, H, d] prologue inputs (raw K; V).
+ * k8, v8, *_scale   : the prologue's FP8 output for K and V.
+ * p                 : the prologue parameters used (positions, k_norm_w, eps).
+ * m                 : tokens to repair per (b, h), 0 <= m <= N.
+ * err               : fp32 [B, H, N] output, e_t above (fp32 arithmetic).
+ * idx               : int32 [B, H, m] output, the m largest e_t of each
+ *                     (b, h) (ties to the lower token), in token order.
+ * k_sel, v_sel      : bf16 [B, H, m, d] outputs, the exact K' and V rows of
+ *                     the selected tokens.
+ * idx, k_sel, v_sel may be NULL when m == 0.  Sizes as jattn_prologue;
+ * 16-byte aligned tensors, 4-byte aligned scales, err and idx.
+ */
+JATTN_API int jattn_fp8_repair_select(const void* k, const void* v, const void* k8, const void* v8,
+                            const float* k_scale, const float* v_scale, const jattn_prologue_params* p,
+                            int m, float* err, int* idx, void* k_sel, void* v_sel,
+                            int B, int H, int N_txt, int N_img, int N_ref, int d, void* cuda_stream);
+
+/*
+ * jattn_fp8_repair_apply — correct jattn_fwd_fp8's O and LSE in place for
+ * the selected keys.
+ *
+ * q8, q_scale, k8, v8, k_scale, v_scale : the FP8 attention's inputs.
+ * idx, k_sel, v_sel, m : jattn_fp8_repair_select's outputs.
+ * o, lse : jattn_fwd_fp8's outputs (lse is required), overwritten with
+ *          attention in which the selected keys use their exact rows:
+ *          with a = sum over them of exp(s_x - L) v_x - exp(s_q - L) v_q and
+ *          z the same sum without v, O' = (O + a) / (1 + z), L' = L + ln(1+z),
+ *          s_x = scale qd.k'_t and s_q = scale qd.kd_t (tensor-core products
+ *          of FP16 operands, fp32 accumulation).
+ * m == 0 leaves o and lse unchanged.  softmax_scale as for jattn_fwd_fp8.
+ */
+JATTN_API int jattn_fp8_repair_apply(const void* q8, const float* q_scale, const void* k8, const void* v8,
+                           const float* k_scale, const float* v_scale, const int* idx,
+                           const void* k_sel, const void* v_sel, int m, void* o, float* lse,
+                           int B, int H, int N_txt, int N_img, int N_ref, int d, float softmax_scale,
+                           void* cuda_stream);
+
 /* Human-readable name of a jattn_status value (static string, never NULL). */
 JATTN_API const char* jattn_status_string(int status);
 
