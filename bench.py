@@ -283,6 +283,29 @@ def time_fp8_path(J, dev, stream, rank: int, peaks, peaks_src, steps: int = 10):
         raise RuntimeError("device error word set during FP8 timing")
     pro = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     att = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # Repair budget rho = 0.005 on top of the FP8 attention: selection
+    # (errors, top-m, exact rows) and the correction, timed separately.
+    m = J.repair_count(w.N, 0.005)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    err = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, w.H, m), dtype=torch.int32, device=dev)
+    ksel = torch.empty((w.B, w.H, m, w.d), dtype=torch.bfloat16, device=dev)
+    vsel = torch.empty_like(ksel)
+    J.jattn_fwd_fp8(q8, k8, v8, qs, ks, vs, o, lse, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d, w.softmax_scale, h)
+    rev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for e in rev:
+        e[0].record(stream)
+        J.jattn_fp8_repair_select(k, v, k8, v8, ks, vs, params, m, err, idx, ksel, vsel, w.B, w.H, w.n_txt,
+                                  w.n_img, w.n_ref, w.d, h)
+        e[1].record(stream)
+        J.jattn_fp8_repair_apply(q8, qs, k8, v8, ks, vs, idx, ksel, vsel, m, o, lse, w.B, w.H, w.n_txt, w.n_img,
+                                 w.n_ref, w.d, w.softmax_scale, h)
+        e[2].record(stream)
+    torch.cuda.synchronize(dev)
+    if J.jattn_device_status(h) != J.JATTN_OK:
+        raise RuntimeError("device error word set during repair timing")
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in rev)
+    app_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in rev)
     fp8_peak = 2.0 * peaks["bf16_tflops"]  # nominal dense fp8 : bf16 ratio 2
     achieved = w.flops / (att * 1e-3) / 1e12
     pro_bytes = w.B * w.N * w.H * w.d * (3 * 2 + 3 * 1) + 3 * w.B * w.H * nblk * 4
@@ -297,6 +320,8 @@ def time_fp8_path(J, dev, stream, rank: int, peaks, peaks_src, steps: int = 10):
         "prologue_roofline": {"bound": "hbm", "achieved": pro_bytes / (pro * 1e-3) / 1e9,
                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": pro_bytes / (pro * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "repair": {"rho": 0.005, "tokens_per_head": m, "select_ms": sel_ms, "apply_ms": app_ms,
+                   "note": "per-token K'/V quantisation error, top-m per head, exact rows, LSE correction"},
     }
 
 

@@ -214,10 +214,26 @@ repair_gather_kernel(const __grid_constant__ PrologueArgs a, const int* __restri
 }
 
 // ----------------------------------------------------------- 4. apply ----
-constexpr int kApplyQ = 64;      // query rows per CTA (one FP8 scale block)
-constexpr int kChunk = 32;       // selected keys per shared-memory chunk
+// CTA = 8 warps x 16 query rows = 128 query rows (two FP8 scale blocks) per
+// pass.  The selected keys are staged in shared memory as FP16, up to
+// kStageMax at a time: when they all fit, a CTA stages them once and walks a
+// run of passes (about one CTA per SM over the grid); otherwise each CTA
+// takes one pass and restages per group of kStageMax keys.
+constexpr int kApplyWarps = 8;
+constexpr int kApplyQ = kApplyWarps * 16;  // query rows per pass
+constexpr int kStageMax = 128;             // selected keys staged at a time
 constexpr int kKStride = kD + 8;         // fp16 per K row (bank-conflict padding)
-constexpr int kVStride = kChunk + 8;     // fp16 per transposed V row
+constexpr int kVStride = kStageMax + 8;  // fp16 per transposed V row
+
+struct ApplySmem {
+  uint8_t q[kApplyQ][kD];                // Q codes of the current query block
+  __half kx[kStageMax][kKStride];        // exact K' (fp16)
+  __half kq[kStageMax][kKStride];        // K codes (fp16)
+  __half vx[kD][kVStride];               // exact V, transposed
+  __half vq[kD][kVStride];               // V codes, transposed
+  float ks[kStageMax], vs[kStageMax];
+};
+constexpr int kApplySmemBytes = static_cast<int>(sizeof(ApplySmem)) + 128;
 
 struct ApplyParams {
   const uint8_t* q8;
@@ -232,6 +248,7 @@ struct ApplyParams {
   __nv_bfloat16* o;
   float* lse;
   int H, N, m;
+  int passes_per_cta;
   float scale_log2;
 };
 
@@ -248,167 +265,183 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-__global__ void __launch_bounds__(128)
-repair_apply_kernel(const __grid_constant__ ApplyParams p) {
-  __shared__ __align__(16) uint8_t s_q[kApplyQ][kD];            // Q codes of the CTA's rows
-  __shared__ __align__(16) __half s_kx[kChunk][kKStride];        // exact K' (fp16)
-  __shared__ __align__(16) __half s_kq[kChunk][kKStride];        // K codes (fp16)
-  __shared__ __align__(16) __half s_vx[kD][kVStride];            // exact V, transposed
-  __shared__ __align__(16) __half s_vq[kD][kVStride];            // V codes, transposed
-  __shared__ float s_ks[kChunk], s_vs[kChunk];
+// Stage selected keys [i0, i0 + n) of (b, h) into shared memory (FP16),
+// zero-padding up to a multiple of 32.
+__device__ __forceinline__ void stage_keys(const ApplyParams& p, ApplySmem& sm, int b, int h, size_t bh, int nblk,
+                                           int i0, int n) {
+  const int n32 = (n + 31) & ~31;
+  for (int e = threadIdx.x; e < n32 * (kD / 8); e += blockDim.x) {
+    const int i = e / (kD / 8), c8 = (e % (kD / 8)) * 8;
+    uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
+    uint2 kc = make_uint2(0, 0), vc = kc;
+    if (i < n) {
+      const size_t sr = (bh * p.m + i0 + i) * kD + c8;
+      kx = __ldg(reinterpret_cast<const uint4*>(p.k_sel + sr));
+      vx = __ldg(reinterpret_cast<const uint4*>(p.v_sel + sr));
+      const int t = __ldg(p.idx + bh * p.m + i0 + i);
+      const size_t cr = ((static_cast<size_t>(b) * p.N + t) * p.H + h) * kD + c8;
+      kc = __ldg(reinterpret_cast<const uint2*>(p.k8 + cr));
+      vc = __ldg(reinterpret_cast<const uint2*>(p.v8 + cr));
+      if (c8 == 0) {
+        sm.ks[i] = __ldg(p.k_scale + bh * nblk + t / kQuantBlock);
+        sm.vs[i] = __ldg(p.v_scale + bh * nblk + t / kQuantBlock);
+      }
+    } else if (c8 == 0) {
+      sm.ks[i] = 0.f;
+      sm.vs[i] = 0.f;
+    }
+    const uint32_t kxw[4] = {kx.x, kx.y, kx.z, kx.w}, vxw[4] = {vx.x, vx.y, vx.z, vx.w};
+    const uint32_t kcw[2] = {kc.x, kc.y}, vcw[2] = {vc.x, vc.y};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      *reinterpret_cast<uint32_t*>(&sm.kx[i][c8 + 2 * j]) = bf16x2_to_f16x2(kxw[j]);
+      *reinterpret_cast<uint32_t*>(&sm.kq[i][c8 + 2 * j]) = e4m3x2_to_f16x2(kcw[j >> 1] >> (16 * (j & 1)));
+      const uint32_t v2 = bf16x2_to_f16x2(vxw[j]);
+      const uint32_t vq2 = e4m3x2_to_f16x2(vcw[j >> 1] >> (16 * (j & 1)));
+      sm.vx[c8 + 2 * j][i] = *reinterpret_cast<const __half*>(&v2);
+      sm.vx[c8 + 2 * j + 1][i] = *(reinterpret_cast<const __half*>(&v2) + 1);
+      sm.vq[c8 + 2 * j][i] = *reinterpret_cast<const __half*>(&vq2);
+      sm.vq[c8 + 2 * j + 1][i] = *(reinterpret_cast<const __half*>(&vq2) + 1);
+    }
+  }
+}
 
+__global__ void __launch_bounds__(kApplyWarps * 32, 1)
+repair_apply_kernel(const __grid_constant__ ApplyParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  ApplySmem& sm = *reinterpret_cast<ApplySmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
   const int h = blockIdx.y, b = blockIdx.z;
-  const int q0 = blockIdx.x * kApplyQ;
   const int N = p.N, H = p.H, m = p.m;
   const int nblk = (N + kQuantBlock - 1) / kQuantBlock;
   const size_t bh = static_cast<size_t>(b) * H + h;
-
-  // Q codes of rows q0 .. q0 + 63 (zero past N).
-  for (int e = threadIdx.x; e < kApplyQ * (kD / 16); e += blockDim.x) {
-    const int rr = e / (kD / 16), cc = e % (kD / 16);
-    const int q = q0 + rr;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (q < N) v = __ldg(reinterpret_cast<const uint4*>(p.q8 + ((static_cast<size_t>(b) * N + q) * H + h) * kD) + cc);
-    *reinterpret_cast<uint4*>(&s_q[rr][cc * 16]) = v;
-  }
-  __syncthreads();
-  // A fragments (16 query rows of this warp x 128 channels) as FP16 codes.
-  uint32_t qa[kD / 16][4];
-  {
-    const int ra = warp * 16 + g, rb = ra + 8;
-#pragma unroll
-    for (int ks = 0; ks < kD / 16; ++ks) {
-      const int c0 = ks * 16 + 2 * tq;
-      qa[ks][0] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&s_q[ra][c0]));
-      qa[ks][1] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&s_q[rb][c0]));
-      qa[ks][2] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&s_q[ra][c0 + 8]));
-      qa[ks][3] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&s_q[rb][c0 + 8]));
-    }
-  }
-  const float qsc = __ldg(p.q_scale + bh * nblk + q0 / kQuantBlock);
-  const int row_a = q0 + warp * 16 + g, row_b = row_a + 8;
+  const bool staged_once = m <= kStageMax;
+  const int npass = (N + kApplyQ - 1) / kApplyQ;
+  const int qb0 = blockIdx.x * p.passes_per_cta;
+  const int qb1 = min(qb0 + p.passes_per_cta, npass);
   const float log2e = 1.4426950408889634f;
-  const float l2a = row_a < N ? __ldg(p.lse + bh * N + row_a) * log2e : 0.f;
-  const float l2b = row_b < N ? __ldg(p.lse + bh * N + row_b) * log2e : 0.f;
-  const float sx = qsc * p.scale_log2;         // exact keys: scale * qd . k'
-  float acc[kD / 8][4];
-#pragma unroll
-  for (int n = 0; n < kD / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  float za = 0.f, zb = 0.f;                    // sum exp(s_x - L) - exp(s_q - L), rows a, b
 
-#pragma unroll 1
-  for (int i0 = 0; i0 < m; i0 += kChunk) {
+  if (staged_once) {
+    stage_keys(p, sm, b, h, bh, nblk, 0, m);
     __syncthreads();
-    // Stage the chunk: exact K' and V rows, K and V codes, their scales.
-    for (int e = threadIdx.x; e < kChunk * (kD / 8); e += blockDim.x) {
-      const int i = e / (kD / 8), c8 = (e % (kD / 8)) * 8;
-      uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
-      uint2 kc = make_uint2(0, 0), vc = kc;
-      if (i0 + i < m) {
-        const size_t sr = (bh * m + i0 + i) * kD + c8;
-        kx = __ldg(reinterpret_cast<const uint4*>(p.k_sel + sr));
-        vx = __ldg(reinterpret_cast<const uint4*>(p.v_sel + sr));
-        const int t = __ldg(p.idx + bh * m + i0 + i);
-        const size_t cr = ((static_cast<size_t>(b) * N + t) * H + h) * kD + c8;
-        kc = __ldg(reinterpret_cast<const uint2*>(p.k8 + cr));
-        vc = __ldg(reinterpret_cast<const uint2*>(p.v8 + cr));
-        if (c8 == 0) {
-          s_ks[i] = __ldg(p.k_scale + bh * nblk + t / kQuantBlock);
-          s_vs[i] = __ldg(p.v_scale + bh * nblk + t / kQuantBlock);
-        }
-      } else if (c8 == 0) {
-        s_ks[i] = 0.f;
-        s_vs[i] = 0.f;
-      }
-      const uint32_t kxw[4] = {kx.x, kx.y, kx.z, kx.w}, vxw[4] = {vx.x, vx.y, vx.z, vx.w};
-      const uint32_t kcw[2] = {kc.x, kc.y}, vcw[2] = {vc.x, vc.y};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        *reinterpret_cast<uint32_t*>(&s_kx[i][c8 + 2 * j]) = bf16x2_to_f16x2(kxw[j]);
-        const uint32_t v2 = bf16x2_to_f16x2(vxw[j]);
-        s_vx[c8 + 2 * j][i] = *reinterpret_cast<const __half*>(&v2);
-        s_vx[c8 + 2 * j + 1][i] = *(reinterpret_cast<const __half*>(&v2) + 1);
-        const uint32_t kq2 = e4m3x2_to_f16x2(kcw[j >> 1] >> (16 * (j & 1)));
-        *reinterpret_cast<uint32_t*>(&s_kq[i][c8 + 2 * j]) = kq2;
-        const uint32_t vq2 = e4m3x2_to_f16x2(vcw[j >> 1] >> (16 * (j & 1)));
-        s_vq[c8 + 2 * j][i] = *reinterpret_cast<const __half*>(&vq2);
-        s_vq[c8 + 2 * j + 1][i] = *(reinterpret_cast<const __half*>(&vq2) + 1);
-      }
+  }
+#pragma unroll 1
+  for (int qb = qb0; qb < qb1; ++qb) {
+    const int q0 = qb * kApplyQ;
+    __syncthreads();  // previous block's readers of sm.q are done
+    for (int e = threadIdx.x; e < kApplyQ * (kD / 16); e += blockDim.x) {
+      const int rr = e / (kD / 16), cc = e % (kD / 16);
+      const int q = q0 + rr;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (q < N) v = __ldg(reinterpret_cast<const uint4*>(p.q8 + ((static_cast<size_t>(b) * N + q) * H + h) * kD) + cc);
+      *reinterpret_cast<uint4*>(&sm.q[rr][cc * 16]) = v;
     }
     __syncthreads();
-
-    // Scores of the 16 rows against the 32 keys, exact and quantised.
-    uint32_t wa[4][4];  // A fragments of [w_x (keys 0-31) | -w_q (keys 0-31)], 4 k-steps of 16
-#pragma unroll
-    for (int nt = 0; nt < kChunk / 8; ++nt) {
-      float cx[4] = {0.f, 0.f, 0.f, 0.f}, cq[4] = {0.f, 0.f, 0.f, 0.f};
-      const int key = nt * 8 + g;  // B column of this lane
+    // A fragments (this warp's 16 query rows x 128 channels), FP16 codes.
+    uint32_t qa[kD / 16][4];
+    {
+      const int ra = warp * 16 + g, rb = ra + 8;
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
         const int c0 = ks * 16 + 2 * tq;
-        mma16816(cx, qa[ks], *reinterpret_cast<const uint32_t*>(&s_kx[key][c0]),
-                 *reinterpret_cast<const uint32_t*>(&s_kx[key][c0 + 8]));
-        mma16816(cq, qa[ks], *reinterpret_cast<const uint32_t*>(&s_kq[key][c0]),
-                 *reinterpret_cast<const uint32_t*>(&s_kq[key][c0 + 8]));
+        qa[ks][0] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&sm.q[ra][c0]));
+        qa[ks][1] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&sm.q[rb][c0]));
+        qa[ks][2] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&sm.q[ra][c0 + 8]));
+        qa[ks][3] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&sm.q[rb][c0 + 8]));
       }
-      // C element j: row (j < 2 ? a : b), key nt*8 + 2 tq + (j & 1).
-      float wx[4], wq[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int kk = nt * 8 + 2 * tq + (j & 1);
-        const bool live = i0 + kk < m;
-        const float l2 = j < 2 ? l2a : l2b;
-        wx[j] = live ? ex2_approx(cx[j] * sx - l2) : 0.f;
-        wq[j] = live ? ex2_approx(cq[j] * (sx * s_ks[kk]) - l2) : 0.f;
-        if (j < 2) za += wx[j] - wq[j]; else zb += wx[j] - wq[j];
-        wq[j] *= s_vs[kk];  // V's block scale folded into the weight
-      }
-      // n-tiles 2k, 2k+1 form the A fragment of k-step k (keys 16k .. 16k+15).
-      const int kstep = nt >> 1, hi = nt & 1;
-      wa[kstep][2 * hi] = pack_h2(wx[0], wx[1]);
-      wa[kstep][2 * hi + 1] = pack_h2(wx[2], wx[3]);
-      wa[2 + kstep][2 * hi] = pack_h2(-wq[0], -wq[1]);
-      wa[2 + kstep][2 * hi + 1] = pack_h2(-wq[2], -wq[3]);
     }
-    // acc += [w_x | -w_q] [V_x ; V_q]
+    const float qsc = __ldg(p.q_scale + bh * nblk + (q0 + warp * 16) / kQuantBlock);
+    const int row_a = q0 + warp * 16 + g, row_b = row_a + 8;
+    const float l2a = row_a < N ? p.lse[bh * N + row_a] * log2e : 0.f;
+    const float l2b = row_b < N ? p.lse[bh * N + row_b] * log2e : 0.f;
+    const float sx = qsc * p.scale_log2;
+    float acc[kD / 8][4];
+#pragma unroll
+    for (int n = 0; n < kD / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    float za = 0.f, zb = 0.f;  // sum exp(s_x - L) - exp(s_q - L), rows a, b
+
+#pragma unroll 1
+    for (int s0 = 0; s0 < m; s0 += kStageMax) {
+      const int ns = min(kStageMax, m - s0);
+      if (!staged_once) {
+        __syncthreads();
+        stage_keys(p, sm, b, h, bh, nblk, s0, ns);
+        __syncthreads();
+      }
+#pragma unroll 1
+      for (int c0k = 0; c0k < ns; c0k += 32) {
+        uint32_t wa[4][4];  // A fragments of [w_x (32 keys) | -w_q (32 keys)]
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          float cx[4] = {0.f, 0.f, 0.f, 0.f}, cq[4] = {0.f, 0.f, 0.f, 0.f};
+          const int key = c0k + nt * 8 + g;  // B column of this lane
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const int cc = ks * 16 + 2 * tq;
+            mma16816(cx, qa[ks], *reinterpret_cast<const uint32_t*>(&sm.kx[key][cc]),
+                     *reinterpret_cast<const uint32_t*>(&sm.kx[key][cc + 8]));
+            mma16816(cq, qa[ks], *reinterpret_cast<const uint32_t*>(&sm.kq[key][cc]),
+                     *reinterpret_cast<const uint32_t*>(&sm.kq[key][cc + 8]));
+          }
+          float wx[4], wq[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int kk = c0k + nt * 8 + 2 * tq + (j & 1);
+            const bool live = kk < ns;
+            const float l2 = j < 2 ? l2a : l2b;
+            wx[j] = live ? ex2_approx(cx[j] * sx - l2) : 0.f;
+            wq[j] = live ? ex2_approx(cq[j] * (sx * sm.ks[kk]) - l2) : 0.f;
+            if (j < 2) za += wx[j] - wq[j]; else zb += wx[j] - wq[j];
+            wq[j] *= sm.vs[kk];  // V's block scale folded into the weight
+          }
+          const int kstep = nt >> 1, hi = nt & 1;
+          wa[kstep][2 * hi] = pack_h2(wx[0], wx[1]);
+          wa[kstep][2 * hi + 1] = pack_h2(wx[2], wx[3]);
+          wa[2 + kstep][2 * hi] = pack_h2(-wq[0], -wq[1]);
+          wa[2 + kstep][2 * hi + 1] = pack_h2(-wq[2], -wq[3]);
+        }
+        // acc += [w_x | -w_q] [V_x ; V_q]
+#pragma unroll
+        for (int n = 0; n < kD / 8; ++n) {
+          const int dcol = n * 8 + g;
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const __half(*vt)[kVStride] = k4 < 2 ? sm.vx : sm.vq;
+            const int kb = c0k + (k4 & 1) * 16 + 2 * tq;
+            mma16816(acc[n], wa[k4], *reinterpret_cast<const uint32_t*>(&vt[dcol][kb]),
+                     *reinterpret_cast<const uint32_t*>(&vt[dcol][kb + 8]));
+          }
+        }
+      }
+    }
+
+    // Row sums over the quad, then O' = (O + a) / (1 + z), L' = L + ln(1 + z).
+    za += __shfl_xor_sync(0xffffffffu, za, 1);
+    za += __shfl_xor_sync(0xffffffffu, za, 2);
+    zb += __shfl_xor_sync(0xffffffffu, zb, 1);
+    zb += __shfl_xor_sync(0xffffffffu, zb, 2);
+    const float ia = 1.f / (1.f + za), ib = 1.f / (1.f + zb);
 #pragma unroll
     for (int n = 0; n < kD / 8; ++n) {
-      const int dcol = n * 8 + g;
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const __half(*vt)[kVStride] = k4 < 2 ? s_vx : s_vq;
-        const int kb = (k4 & 1) * 16 + 2 * tq;
-        mma16816(acc[n], wa[k4], *reinterpret_cast<const uint32_t*>(&vt[dcol][kb]),
-                 *reinterpret_cast<const uint32_t*>(&vt[dcol][kb + 8]));
+      const int c = n * 8 + 2 * tq;
+      if (row_a < N) {
+        __nv_bfloat162* o2 =
+            reinterpret_cast<__nv_bfloat162*>(p.o + ((static_cast<size_t>(b) * N + row_a) * H + h) * kD + c);
+        const float2 f = __bfloat1622float2(*o2);
+        *o2 = __floats2bfloat162_rn((f.x + acc[n][0]) * ia, (f.y + acc[n][1]) * ia);
+      }
+      if (row_b < N) {
+        __nv_bfloat162* o2 =
+            reinterpret_cast<__nv_bfloat162*>(p.o + ((static_cast<size_t>(b) * N + row_b) * H + h) * kD + c);
+        const float2 f = __bfloat1622float2(*o2);
+        *o2 = __floats2bfloat162_rn((f.x + acc[n][2]) * ib, (f.y + acc[n][3]) * ib);
       }
     }
-  }
-
-  // Row sums over the quad, then O' = (O + a) / (1 + z), L' = L + ln(1 + z).
-  za += __shfl_xor_sync(0xffffffffu, za, 1);
-  za += __shfl_xor_sync(0xffffffffu, za, 2);
-  zb += __shfl_xor_sync(0xffffffffu, zb, 1);
-  zb += __shfl_xor_sync(0xffffffffu, zb, 2);
-  const float ia = 1.f / (1.f + za), ib = 1.f / (1.f + zb);
-#pragma unroll
-  for (int n = 0; n < kD / 8; ++n) {
-    const int c = n * 8 + 2 * tq;
-    if (row_a < N) {
-      __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(p.o + ((static_cast<size_t>(b) * N + row_a) * H + h) * kD + c);
-      const float2 f = __bfloat1622float2(*o2);
-      *o2 = __floats2bfloat162_rn((f.x + acc[n][0]) * ia, (f.y + acc[n][1]) * ia);
+    if (tq == 0) {
+      if (row_a < N) p.lse[bh * N + row_a] += __logf(1.f + za);
+      if (row_b < N) p.lse[bh * N + row_b] += __logf(1.f + zb);
     }
-    if (row_b < N) {
-      __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(p.o + ((static_cast<size_t>(b) * N + row_b) * H + h) * kD + c);
-      const float2 f = __bfloat1622float2(*o2);
-      *o2 = __floats2bfloat162_rn((f.x + acc[n][2]) * ib, (f.y + acc[n][3]) * ib);
-    }
-  }
-  if (tq == 0) {
-    if (row_a < N) p.lse[bh * N + row_a] += __logf(1.f + za);
-    if (row_b < N) p.lse[bh * N + row_b] += __logf(1.f + zb);
   }
 }
 
@@ -447,9 +480,16 @@ cudaError_t launch_repair_apply(const RepairProblem& r, int B, int H, int N, flo
   p.H = H;
   p.N = N;
   p.m = r.m;
+  // Keys staged once: about one CTA per SM, each walking a run of passes.
+  const int npass = (N + kApplyQ - 1) / kApplyQ;
+  int per_head = 1;
+  if (r.m <= kStageMax) per_head = std::max(1, std::min(npass, device_sm_count() / std::max(1, B * H)));
+  p.passes_per_cta = r.m <= kStageMax ? (npass + per_head - 1) / per_head : 1;
   p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
-  dim3 grid((N + kApplyQ - 1) / kApplyQ, H, B);
-  repair_apply_kernel<<<grid, 128, 0, s>>>(p);
+  cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(repair_apply_kernel), kApplySmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((npass + p.passes_per_cta - 1) / p.passes_per_cta, H, B);
+  repair_apply_kernel<<<grid, kApplyWarps * 32, kApplySmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 
