@@ -19,7 +19,8 @@ arithmetic.  Sources (titles of the web pages the method is described on):
   projection epilogue applies query/key normalisation and rotary position
   embedding (in that order).
 * "Quantized and sparse attention" section of the same tutorial: FP8 Q/K
-  and FP8 V attention (``qk_dtype: fp8``, ``v_dtype: fp8``).
+  and FP8 V attention (``qk_dtype: fp8``, ``v_dtype: fp8``), the
+  VC-Attention FP8 repair budget and Sol-Attention block sparsity.
 
 The pages fix no constants (head size, eps, RoPE base and axis split, block
 size, quantisation format); those come from the workload definitions and
@@ -29,13 +30,18 @@ the function that applies it.
 Pins: every function here is checked by ``tests/test_oracle_pins.py``
 against closed forms, hand-derived worked values (``tests/golden/``),
 library routines (torch float64 SDPA, ``torch.float8_e4m3fn``) and
-invariants.  No function here is "parity unpinned".
+invariants.  One reading is parity unpinned against the pages: the meaning
+of Sol-Attention's tau (``sparse_probs`` / ``sparse_keep``), which the pages
+name but do not define; the rule implemented is pinned as stated.
 """
 
 from .jattn_oracle import (  # noqa: F401
     E4M3_MAX,
+    SPARSE_KBLOCK,
+    SPARSE_QBLOCK,
     bf16_round,
     bf16_ulp_distance,
+    block_sparse_attention,
     block_quantize_e4m3,
     dequantize_e4m3,
     e4m3_decode,
@@ -49,5 +55,8 @@ from .jattn_oracle import (  # noqa: F401
     rmsnorm,
     rope_2d,
     rope_table,
+    sparse_keep,
+    sparse_pool,
+    sparse_probs,
     token_positions,
 )

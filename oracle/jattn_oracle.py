@@ -390,3 +390,100 @@ def repaired_attention(q_deq, k_deq, v_deq, k_exact, v_exact, idx, scale: float)
             k[b, t, h, :] = np.asarray(k_exact, np.float64)[b, t, h, :]
             v[b, t, h, :] = np.asarray(v_exact, np.float64)[b, t, h, :]
     return joint_attention(q_deq, k, v, scale)
+
+
+# ---------------------------------------------------------------------------
+# Block-sparse attention (Sol-Attention style)
+# ---------------------------------------------------------------------------
+#
+# The tutorial's "Quantized and sparse attention" section runs Sol-Attention
+# through a generic block-sparse attention kernel, with the sparsity set by
+# a parameter tau (tau = 1.0 in its tests; a higher tau lowers quality for
+# little extra speed) and the first denoising steps kept dense.  It does not
+# define tau or the block rule.  Reading used here (parity unpinned against
+# the pages for the meaning of tau; the rule below is pinned as stated):
+#
+#   blocks     query blocks of SPARSE_QBLOCK consecutive joint-sequence
+#              tokens, key blocks of SPARSE_KBLOCK, counted from token 0 of
+#              each (b, h); the last block of each kind may be partial;
+#   pooled     qbar_i, kbar_j = mean of the block's Q' (resp. K') rows;
+#   score      p_ij = softmax_j(scale * qbar_i . kbar_j) over the n_kb key
+#              blocks of the (b, h);
+#   keep       key block j for query block i iff p_ij >= tau / n_kb (at least
+#              tau times the uniform share), and always the block with the
+#              largest p_ij (lowest index among equals), so no row is empty;
+#   attention  each query attends, with an ordinary softmax, to the keys of
+#              its query block's kept key blocks only.
+# tau = 0 keeps every block (dense attention); a larger tau keeps a subset.
+
+SPARSE_QBLOCK = 256
+SPARSE_KBLOCK = 128
+
+
+def sparse_pool(x, block: int) -> np.ndarray:
+    """Mean of ``x[B, N, H, d]`` over consecutive blocks of ``block`` tokens
+    (the last one partial), per (b, h): ``[B, H, ceil(N / block), d]``."""
+    x = np.asarray(x, dtype=np.float64)
+    B, N, H, d = x.shape
+    nb = -(-N // block)
+    out = np.empty((B, H, nb, d), dtype=np.float64)
+    for i in range(nb):
+        out[:, :, i, :] = np.mean(x[:, i * block:min(N, (i + 1) * block)], axis=1)
+    return out
+
+
+def sparse_probs(q, k, scale: float, qblock: int = SPARSE_QBLOCK, kblock: int = SPARSE_KBLOCK) -> np.ndarray:
+    """Pooled block attention ``p [B, H, n_qb, n_kb]`` (float64): row i is
+    softmax_j(scale * qbar_i . kbar_j)."""
+    qb, kb = sparse_pool(q, qblock), sparse_pool(k, kblock)
+    s = float(scale) * np.einsum("bhic,bhjc->bhij", qb, kb)
+    s -= np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def sparse_keep(probs, tau: float) -> np.ndarray:
+    """Kept key blocks ``bool [..., n_qb, n_kb]`` from pooled probabilities.
+
+    The decision is taken in float32, the precision the GPU path computes
+    ``probs`` in: keep iff ``float32(p) >= float32(tau) / float32(n_kb)``
+    (one correctly rounded division), plus the first block of largest p.
+    """
+    p = np.asarray(probs, dtype=np.float32)
+    nkb = p.shape[-1]
+    thr = np.float32(tau) / np.float32(nkb)
+    keep = p >= thr
+    top = np.argmax(p, axis=-1)   # first index of the maximum
+    np.put_along_axis(keep, top[..., None], True, axis=-1)
+    return keep
+
+
+def block_sparse_attention(q, k, v, keep, scale: float, rows=None,
+                           qblock: int = SPARSE_QBLOCK, kblock: int = SPARSE_KBLOCK):
+    """Attention of each query over the keys of its query block's kept key
+    blocks: ``keep[b, h, i, j]`` for query block i = t // qblock and key
+    block j.  A query whose block keeps nothing gets O = 0 and L = -inf.
+    ``rows`` selects query indices as in joint_attention.  Returns
+    ``O [B, R, H, d]`` and ``L [B, H, R]`` (float64)."""
+    B, N, H, d = q.shape
+    idx = np.arange(N) if rows is None else np.asarray(rows)
+    R = len(idx)
+    keep = np.asarray(keep, dtype=bool)
+    out = np.zeros((B, R, H, v.shape[-1]), dtype=np.float64)
+    lse = np.full((B, H, R), -np.inf, dtype=np.float64)
+    sc = float(scale)
+    f64 = lambda a: np.asarray(a, dtype=np.float64)
+    key_block = np.arange(N) // kblock
+    for b in range(B):
+        for h in range(H):
+            for r, t in enumerate(idx):
+                cols = np.nonzero(keep[b, h, t // qblock][key_block])[0]
+                if cols.size == 0:
+                    continue
+                s = sc * (f64(k[b, cols, h, :]) @ f64(q[b, t, h, :]))
+                m = np.max(s)
+                p = np.exp(s - m)
+                l = np.sum(p)
+                out[b, r, h, :] = (p / l) @ f64(v[b, cols, h, :])
+                lse[b, h, r] = m + np.log(l)
+    return out, lse

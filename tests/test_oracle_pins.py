@@ -478,3 +478,121 @@ def test_repaired_attention_limits():
     idx, _ = O.repair_select(ke, ve, kd, vd, rho=0.3)
     oh, _ = O.repaired_attention(qd, kd, vd, ke, ve, idx, 0.09)
     assert np.linalg.norm(oh - r1) < np.linalg.norm(o0 - r1)
+
+
+# -------------------------------------------------------- block sparse ----
+
+def test_sparse_pool_block_means_of_a_ramp():
+    # x[b, t, h, c] = t + 100 h: the mean of a block [a, e) is (a + e - 1) / 2.
+    N, H = 11, 2
+    x = np.zeros((1, N, H, 3))
+    for h in range(H):
+        x[0, :, h, :] = (np.arange(N) + 100 * h)[:, None]
+    pooled = O.sparse_pool(x, 4)
+    assert pooled.shape == (1, H, 3, 3)
+    for h in range(H):
+        np.testing.assert_allclose(pooled[0, h, :, 0], np.array([1.5, 5.5, 9.0]) + 100 * h)
+
+
+def _hand_sparse_case():
+    # Query rows all e0; key block j (2 tokens) rows ln(j + 1) e0; scale 1:
+    # pooled scores ln(j + 1), so p_ij = (j + 1) / 10 for every query block.
+    N, d = 8, 4
+    q = np.zeros((1, N, 1, d))
+    k = np.zeros((1, N, 1, d))
+    q[0, :, 0, 0] = 1.0
+    for j in range(4):
+        k[0, 2 * j:2 * j + 2, 0, 0] = math.log(j + 1)
+    return q, k
+
+
+def test_sparse_probs_hand_case():
+    q, k = _hand_sparse_case()
+    p = O.sparse_probs(q, k, 1.0, qblock=2, kblock=2)
+    assert p.shape == (1, 1, 4, 4)
+    np.testing.assert_allclose(p, np.broadcast_to([0.1, 0.2, 0.3, 0.4], p.shape), rtol=1e-12)
+
+
+@pytest.mark.parametrize("tau,kept", [(0.0, [0, 1, 2, 3]), (0.5, [1, 2, 3]), (1.0, [2, 3]), (2.0, [3]),
+                                      (9.0, [3])])
+def test_sparse_keep_hand_case(tau, kept):
+    # Threshold tau / 4 against p = (0.1, 0.2, 0.3, 0.4); the top block always stays.
+    q, k = _hand_sparse_case()
+    keep = O.sparse_keep(O.sparse_probs(q, k, 1.0, qblock=2, kblock=2), tau)
+    for i in range(4):
+        assert np.nonzero(keep[0, 0, i])[0].tolist() == kept
+
+
+def test_sparse_keep_ties_take_the_first_maximum():
+    keep = O.sparse_keep(np.array([[0.25, 0.375, 0.375]]), 5.0)
+    assert keep.tolist() == [[False, True, False]]
+
+
+def test_sparse_keep_monotone_in_tau():
+    rng = np.random.default_rng(3)
+    p = rng.dirichlet(np.ones(37), size=(2, 3, 5))
+    k0, k1, k2 = (O.sparse_keep(p, t) for t in (0.5, 1.0, 2.0))
+    assert not (k1 & ~k0).any() and not (k2 & ~k1).any()
+    assert O.sparse_keep(p, 0.0).all()
+    top = np.argmax(p, axis=-1)
+    assert np.take_along_axis(k2, top[..., None], axis=-1).all()
+
+
+def _brute_block_sparse(q, k, v, keep, scale, qblock, kblock):
+    # Naive loops: collect each query's keys one by one, softmax with math.exp.
+    B, N, H, d = q.shape
+    out = np.zeros((B, N, H, d))
+    lse = np.full((B, H, N), -math.inf)
+    for b in range(B):
+        for h in range(H):
+            for t in range(N):
+                keys = [u for u in range(N) if keep[b, h, t // qblock, u // kblock]]
+                if not keys:
+                    continue
+                s = [scale * sum(q[b, t, h, c] * k[b, u, h, c] for c in range(d)) for u in keys]
+                m = max(s)
+                w = [math.exp(x - m) for x in s]
+                tot = sum(w)
+                for c in range(d):
+                    out[b, t, h, c] = sum(wi * v[b, u, h, c] for wi, u in zip(w, keys)) / tot
+                lse[b, h, t] = m + math.log(tot)
+    return out, lse
+
+
+def test_block_sparse_attention_brute_force():
+    rng = np.random.default_rng(4)
+    B, N, H, d = 1, 11, 2, 3
+    q, k, v = (rng.standard_normal((B, N, H, d)) for _ in range(3))
+    keep = rng.random((B, H, 4, 3)) < 0.5       # query blocks of 3, key blocks of 4
+    keep[0, 0, 1] = False                       # one query block with no keys
+    keep[0, 1, 2] = [False, False, True]        # only the partial last key block
+    got, glse = O.block_sparse_attention(q, k, v, keep, 0.7, qblock=3, kblock=4)
+    ref, rlse = _brute_block_sparse(q, k, v, keep, 0.7, 3, 4)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+    np.testing.assert_array_equal(np.isinf(glse), np.isinf(rlse))
+    fin = np.isfinite(rlse)
+    np.testing.assert_allclose(glse[fin], rlse[fin], rtol=1e-12)
+    assert np.all(got[0, 3:6, 0] == 0.0)
+
+
+def test_block_sparse_attention_all_kept_is_joint_attention():
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.standard_normal((2, 70, 2, 8)) for _ in range(3))
+    keep = O.sparse_keep(O.sparse_probs(q, k, 0.3, qblock=32, kblock=16), 0.0)
+    assert keep.all()
+    got, glse = O.block_sparse_attention(q, k, v, keep, 0.3, qblock=32, kblock=16)
+    ref, rlse = O.joint_attention(q, k, v, 0.3)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(glse, rlse, rtol=1e-12)
+    rows = np.array([0, 31, 32, 69])
+    sub, slse = O.block_sparse_attention(q, k, v, keep, 0.3, rows=rows, qblock=32, kblock=16)
+    np.testing.assert_allclose(sub, ref[:, rows], rtol=1e-12, atol=1e-13)
+
+
+def test_block_sparse_attention_of_constant_values_is_constant():
+    rng = np.random.default_rng(6)
+    q, k = (rng.standard_normal((1, 40, 1, 4)) for _ in range(2))
+    v = np.ones((1, 40, 1, 4)) * 2.5
+    keep = O.sparse_keep(O.sparse_probs(q, k, 0.5, qblock=16, kblock=8), 1.0)
+    got, _ = O.block_sparse_attention(q, k, v, keep, 0.5, qblock=16, kblock=8)
+    np.testing.assert_allclose(got, 2.5, rtol=1e-13)
