@@ -30,6 +30,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from diffusion_transformer_joint_dit_b200 import inputs as I  # noqa: E402
@@ -55,6 +56,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-path timing object")
     ap.add_argument("--no-qkv", action="store_true", help="skip the fused-QKV-projection timing object")
+    ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse attention timing object")
     ap.add_argument("--sp", action="store_true",
                     help="Ulysses sequence parallelism over all ranks (strong scaling of one problem) "
                          "instead of one independent problem per rank")
@@ -325,6 +327,71 @@ def time_fp8_path(J, dev, stream, rank: int, peaks, peaks_src, steps: int = 10):
     }
 
 
+def time_sparse_path(J, dev, stream, rank: int, peaks, peaks_src, dense_ms: float, steps: int = 10):
+    """Block-sparse attention (Sol-Attention reading, tau = 1.0) on the
+    t2i_2048 workload: jattn_prologue (BF16), jattn_sparse_select (pooled
+    block scores, kept-block lists), jattn_fwd_bf16_sparse.  The work is the
+    kept (query, key) pairs: 4 d per pair, counted from the lists.  Reported
+    beside the headline line, not instead of it."""
+    w = I.WORKLOADS["t2i_2048"]
+    tau = 1.0
+    q, k, v = (t.to(dev) for t in I.make_qkv(w, seed=rank))
+    params = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps)
+    h = stream.cuda_stream
+    J.jattn_prologue(q, k, None, q, k, None, None, None, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+                     J.JATTN_PROLOGUE_BF16, params, h)
+    nqb, nkb = J.sparse_blocks(w.N)
+    qbar = torch.empty((w.B, w.H, nqb, w.d), dtype=torch.float32, device=dev)
+    kbar = torch.empty((w.B, w.H, nkb, w.d), dtype=torch.float32, device=dev)
+    idx = torch.empty((w.B, w.H, nqb, nkb), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.B, w.H, nqb), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        J.jattn_sparse_select(q, k, qbar, kbar, None, idx, cnt, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+                              w.softmax_scale, tau, h)
+        if ev is not None:
+            ev[1].record(stream)
+        J.jattn_fwd_bf16_sparse(q, k, v, o, None, idx, cnt, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+                                w.softmax_scale, h)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(3):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for e in evs:
+        step(e)
+    torch.cuda.synchronize(dev)
+    if J.jattn_device_status(h) != J.JATTN_OK:
+        raise RuntimeError("device error word set during sparse timing")
+    sel = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    # Kept (query, key) pairs, from the lists (outside the timed region).
+    ci, ii = cnt.cpu().numpy(), idx.cpu().numpy()
+    qrows = np.minimum(w.N - np.arange(nqb) * J.JATTN_SPARSE_QBLOCK, J.JATTN_SPARSE_QBLOCK)
+    kcols = np.minimum(w.N - np.arange(nkb) * J.JATTN_SPARSE_KBLOCK, J.JATTN_SPARSE_KBLOCK)
+    pairs = 0
+    for pos in np.ndindex(*ci.shape):
+        pairs += int(qrows[pos[-1]]) * int(kcols[ii[pos][:ci[pos]]].sum())
+    flops = 4.0 * pairs * w.d
+    achieved = flops / (att * 1e-3) / 1e12
+    return {
+        "workload": f"t2i_2048 block-sparse: B={w.B} H={w.H} N={w.N} d={w.d}, tau={tau}, query blocks "
+                    f"{J.JATTN_SPARSE_QBLOCK}, key blocks {J.JATTN_SPARSE_KBLOCK}",
+        "steps": steps, "select_ms": sel, "attention_ms": att,
+        "kept_fraction": pairs / (w.B * w.H * w.N * w.N), "flops_per_launch": flops,
+        "value": achieved, "unit": UNIT,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "peak_source": f"{peaks_src} bf16_tflops"},
+        "speedup_vs_dense_attention": dense_ms / (sel + att),
+        "note": "synthetic N(0,1) inputs after the prologue; kept fraction is data dependent",
+    }
+
+
 def time_qkv_fused(J, dev, stream, rank: int, peaks, peaks_src, steps: int = 10):
     """Fused QKV projection (RMSNorm + RoPE in the GEMM epilogue) on the
     t2i_2048 shapes: x [B, N, C = H d] -> Q, K, V [B, N, H, d], per-stream
@@ -572,6 +639,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         line["fp8_path"] = time_fp8_path(J, dev, stream, rank, peaks, peaks_src)
     if not args.no_qkv:
         line["qkv_fused"] = time_qkv_fused(J, dev, stream, rank, peaks, peaks_src)
+    if not args.no_sparse:
+        line["sparse_path"] = time_sparse_path(J, dev, stream, rank, peaks, peaks_src, att_ms)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k_: v_ for k_, v_ in cpu_baseline(w, q, k, v, args.cpu_seconds).items()
                                 if k_ != "seconds"}

@@ -26,9 +26,11 @@ JATTN_ERR_TIMEOUT = 5
 JATTN_PROLOGUE_BF16 = 0
 JATTN_PROLOGUE_FP8 = 1
 JATTN_FP8_BLOCK = 64
+JATTN_SPARSE_QBLOCK = 256
+JATTN_SPARSE_KBLOCK = 128
 
 EXPORTED = ("jattn_prologue", "jattn_fwd_bf16", "jattn_fwd_fp8", "jattn_rope_table", "jattn_qkv_fused",
-            "jattn_fp8_repair_select", "jattn_fp8_repair_apply",
+            "jattn_fp8_repair_select", "jattn_fp8_repair_apply", "jattn_sparse_select", "jattn_fwd_bf16_sparse",
             "jattn_status_string", "jattn_device_status", "jattn_selftest_wait_timeout",
             "jattn_selftest_exp2_poly", "jattn_last_cuda_error")
 
@@ -93,6 +95,11 @@ def load_library():
     lib.jattn_fp8_repair_apply.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P,
                                            _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]
     lib.jattn_fp8_repair_apply.restype = _I
+    lib.jattn_sparse_select.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                        ctypes.c_float, ctypes.c_float, _P]
+    lib.jattn_sparse_select.restype = _I
+    lib.jattn_fwd_bf16_sparse.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]
+    lib.jattn_fwd_bf16_sparse.restype = _I
     lib.jattn_status_string.argtypes = [_I]
     lib.jattn_status_string.restype = ctypes.c_char_p
     lib.jattn_device_status.argtypes = [_P]
@@ -230,6 +237,32 @@ def jattn_fp8_repair_apply(q8, q_scale, k8, v8, k_scale, v_scale, idx, k_sel, v_
         _ptr(v_sel), m, _ptr(o), _ptr(lse), B, H, N_txt, N_img, N_ref, d, softmax_scale, _stream(stream))
     if check:
         _check("jattn_fp8_repair_apply", st)
+    return st
+
+
+def sparse_blocks(n: int) -> tuple:
+    """(query blocks, key blocks) of a joint sequence of n tokens."""
+    return -(-n // JATTN_SPARSE_QBLOCK), -(-n // JATTN_SPARSE_KBLOCK)
+
+
+def jattn_sparse_select(q, k, qbar, kbar, probs, kv_idx, kv_cnt, B: int, H: int, N_txt: int, N_img: int,
+                        N_ref: int, d: int, softmax_scale: float, tau: float, stream=None, *,
+                        check: bool = True) -> int:
+    st = load_library().jattn_sparse_select(
+        _ptr(q), _ptr(k), _ptr(qbar), _ptr(kbar), _ptr(probs), _ptr(kv_idx), _ptr(kv_cnt),
+        B, H, N_txt, N_img, N_ref, d, softmax_scale, tau, _stream(stream))
+    if check:
+        _check("jattn_sparse_select", st)
+    return st
+
+
+def jattn_fwd_bf16_sparse(q, k, v, o, lse, kv_idx, kv_cnt, B: int, H: int, N_txt: int, N_img: int, N_ref: int,
+                          d: int, softmax_scale: float, stream=None, *, check: bool = True) -> int:
+    st = load_library().jattn_fwd_bf16_sparse(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(kv_idx), _ptr(kv_cnt),
+        B, H, N_txt, N_img, N_ref, d, softmax_scale, _stream(stream))
+    if check:
+        _check("jattn_fwd_bf16_sparse", st)
     return st
 
 

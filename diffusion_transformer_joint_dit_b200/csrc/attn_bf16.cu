@@ -31,6 +31,13 @@
 // The O rescale (a TMEM read-modify-write) is thus rare after the first
 // tiles.  Tail keys (N not a multiple of 128) are masked to -inf; tail
 // query rows read zero-filled Q and are not stored.
+//
+// Block-sparse variant (kSparse): the tutorial's Sol-Attention runs a
+// generic block-sparse attention kernel.  A CTA's 256 query rows are one
+// query block; it visits only the KV tiles listed for that block (a count
+// and increasing tile indices per (b, h, query block)) instead of all of
+// them, with the same pipeline.  A block with an empty list writes O = 0
+// and LSE = -inf.
 #include "jattn_internal.h"
 #include "sm100_ptx.cuh"
 #include "softmax_sm100.cuh"
@@ -78,6 +85,8 @@ constexpr int kSmemBytes = kSmemCtrl + static_cast<int>(sizeof(Ctrl)) + 1024;  /
 struct Params {
   __nv_bfloat16* o;
   float* lse;
+  const int* kv_idx;  // block-sparse only: [B, H, n_qb, n_kv] tile lists
+  const int* kv_cnt;  // block-sparse only: [B, H, n_qb] list lengths
   int H, N;
   float scale_log2;
   uint64_t timeout_ns;
@@ -89,6 +98,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint6
   return mbar_wait(bar, parity, &never, timeout_ns);
 }
 
+template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params prm) {
@@ -104,6 +114,19 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int m0 = blockIdx.x * (kBM * kTiles);
   const int N = prm.N;
   const int n_kv = (N + kBN - 1) / kBN;
+  // KV tiles visited: all of them, or the query block's list.
+  const int* list = nullptr;
+  int n_iter = n_kv;
+  if constexpr (kSparse) {
+    const size_t blk = (static_cast<size_t>(b) * prm.H + h) * gridDim.x + blockIdx.x;
+    list = prm.kv_idx + blk * n_kv;
+    n_iter = min(max(__ldg(prm.kv_cnt + blk), 0), n_kv);
+  }
+  // Tile of the jj-th visit (clamped into range: memory-safe for any list).
+  auto tile_of = [&](int jj) -> int {
+    if constexpr (kSparse) return min(max(__ldg(list + jj), 0), n_kv - 1);
+    return jj;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
@@ -143,7 +166,8 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       int it = 0;
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
+      for (int jj = 0; jj < n_iter && ok; ++jj) {
+        const int j = tile_of(jj);
         for (int which = 0; which < 2; ++which, ++it) {
           const int slot = it % kStages;
           const uint32_t round = static_cast<uint32_t>(it / kStages);
@@ -198,8 +222,8 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
       bool ok = mbar_wait(&ctrl->q_full, 0, abort_flag, prm.timeout_ns);
       int it = 0;
-      if (ok) ok = mbar_wait(&ctrl->kv_full[0], 0, abort_flag, prm.timeout_ns);
-      if (ok) {
+      if (ok && n_iter > 0) ok = mbar_wait(&ctrl->kv_full[0], 0, abort_flag, prm.timeout_ns);
+      if (ok && n_iter > 0) {
         tc_fence_after();
         issue_qk(0, 0);
         mma_commit(&ctrl->s_full[0]);
@@ -208,13 +232,13 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mma_commit(&ctrl->kv_empty[0]);
         it = 1;
       }
-      for (int j = 0; j < n_kv && ok; ++j) {
+      for (int j = 0; j < n_iter && ok; ++j) {
         const int slot_v = it % kStages;
         ok = mbar_wait(&ctrl->kv_full[slot_v], static_cast<uint32_t>(it / kStages) & 1u, abort_flag,
                        prm.timeout_ns);
         ++it;
         if (!ok) break;
-        const bool has_next = j + 1 < n_kv;
+        const bool has_next = j + 1 < n_iter;
         const int slot_k = it % kStages;
         // Q tile 0
         ok = mbar_wait(&ctrl->p_full[0], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns);
@@ -261,7 +285,8 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float m = -INFINITY;  // reference row max (log2 units of scaled logits)
     float l = 0.f;        // row sum of exp2(x - m)
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; j < n_iter; ++j) {
+      const int tile = tile_of(j);  // issued before the wait: its latency hides there
       // Warp-uniform outcome: the tcgen05.ld/st below are warp-collective.
       if (!__all_sync(0xffffffffu,
                       mbar_wait(&ctrl->s_full[t], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns))) {
@@ -275,7 +300,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_wait(sv[c]);  // ties the loaded registers to the wait
 
-      const int nvalid = N - j * kBN;  // >= 1
+      const int nvalid = N - tile * kBN;  // >= 1
       if (nvalid < kBN) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -321,13 +346,21 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->o_full, 0, abort_flag, prm.timeout_ns))) {
       tc_fence_after();
       const int row = m0 + t * kBM + r;
-      const float inv_l = 1.0f / l;
+      // l > 0 whenever a tile was visited (the row max contributes 1).
+      const bool empty = kSparse && !(l > 0.f);
+      const float inv_l = empty ? 0.f : 1.0f / l;
       __nv_bfloat16* orow = prm.o + ((static_cast<size_t>(b) * N + row) * prm.H + h) * kD;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t ov[32];
         tmem_ld32(o_addr + c * 32, ov);
         tmem_ld_wait(ov);
+        if constexpr (kSparse) {
+          if (empty) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = 0u;  // O's columns were never written
+          }
+        }
         if (row < N) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
@@ -342,7 +375,8 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       }
       if (prm.lse != nullptr && row < N) {
-        prm.lse[(static_cast<size_t>(b) * prm.H + h) * N + row] = (m + __log2f(l)) * 0.69314718055994530942f;
+        prm.lse[(static_cast<size_t>(b) * prm.H + h) * N + row] =
+            empty ? -INFINITY : (m + __log2f(l)) * 0.69314718055994530942f;
       }
     }
   }
@@ -358,24 +392,40 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 }  // namespace bf16attn
 
 
-cudaError_t launch_attn_bf16(const AttnProblem& p, cudaStream_t s) {
+namespace {
+
+template <bool kSparse>
+cudaError_t launch_bf16(const AttnProblem& p, const int* kv_idx, const int* kv_cnt, cudaStream_t s) {
   using namespace bf16attn;
   CUtensorMap tq, tk, tv;
   cudaError_t e;
   if ((e = make_act_map(&tq, p.q, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
   if ((e = make_act_map(&tk, p.k, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
   if ((e = make_act_map(&tv, p.v, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
-  if ((e = set_smem_attr(reinterpret_cast<const void*>(attn_bf16_kernel), kSmemBytes)) != cudaSuccess) return e;
+  if ((e = set_smem_attr(reinterpret_cast<const void*>(attn_bf16_kernel<kSparse>), kSmemBytes)) != cudaSuccess)
+    return e;
   Params prm;
   prm.o = static_cast<__nv_bfloat16*>(p.o);
   prm.lse = p.lse;
+  prm.kv_idx = kv_idx;
+  prm.kv_cnt = kv_cnt;
   prm.H = p.H;
   prm.N = p.N;
   prm.scale_log2 = static_cast<float>(static_cast<double>(p.softmax_scale) * 1.4426950408889634074);
   prm.timeout_ns = p.timeout_ns;
   dim3 grid((p.N + kBM * kTiles - 1) / (kBM * kTiles), p.H, p.B);
-  attn_bf16_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, prm);
+  attn_bf16_kernel<kSparse><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, prm);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_bf16(const AttnProblem& p, cudaStream_t s) {
+  return launch_bf16<false>(p, nullptr, nullptr, s);
+}
+
+cudaError_t launch_attn_bf16_sparse(const AttnProblem& p, const int* kv_idx, const int* kv_cnt, cudaStream_t s) {
+  return launch_bf16<true>(p, kv_idx, kv_cnt, s);
 }
 
 }  // namespace jattn

@@ -17,6 +17,7 @@
 #include "qkv_gemm.cu"
 #include "prologue.cu"
 #include "repair.cu"
+#include "sparse.cu"
 
 namespace jattn {
 
@@ -255,6 +256,51 @@ int jattn_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   pr.softmax_scale = softmax_scale;
   pr.timeout_ns = kDefaultTimeoutNs;
   return map_err(launch_attn_bf16(pr, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+int jattn_sparse_select(const void* q, const void* k, float* qbar, float* kbar, float* probs, int* kv_idx,
+                        int* kv_cnt, int B, int H, int N_txt, int N_img, int N_ref, int d, float softmax_scale,
+                        float tau, void* cuda_stream) {
+  int st = check_common(B, H, N_txt, N_img, N_ref, d);
+  if (st != JATTN_OK) return st;
+  if (q == nullptr || k == nullptr || qbar == nullptr || kbar == nullptr || kv_idx == nullptr || kv_cnt == nullptr)
+    return JATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return JATTN_ERR_INVALID_ARG;
+  if (!(tau >= 0.f) || !std::isfinite(tau)) return JATTN_ERR_INVALID_ARG;
+  const int N = N_txt + N_img + N_ref;
+  if (N > (1 << 22)) return JATTN_ERR_INVALID_ARG;  // key-block scores are staged in shared memory
+  if (!aligned16(q) || !aligned16(k) || !aligned16(qbar) || !aligned16(kbar) ||
+      (reinterpret_cast<uintptr_t>(probs) & 3u) || (reinterpret_cast<uintptr_t>(kv_idx) & 3u) ||
+      (reinterpret_cast<uintptr_t>(kv_cnt) & 3u))
+    return JATTN_ERR_MISALIGNED;
+  SparseProblem sp;
+  std::memset(&sp, 0, sizeof(sp));
+  sp.q = q; sp.k = k; sp.qbar = qbar; sp.kbar = kbar; sp.probs = probs; sp.kv_idx = kv_idx; sp.kv_cnt = kv_cnt;
+  sp.B = B; sp.H = H; sp.N = N;
+  sp.softmax_scale = softmax_scale;
+  sp.tau = tau;
+  return map_err(launch_sparse_select(sp, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+int jattn_fwd_bf16_sparse(const void* q, const void* k, const void* v, void* o, float* lse, const int* kv_idx,
+                          const int* kv_cnt, int B, int H, int N_txt, int N_img, int N_ref, int d,
+                          float softmax_scale, void* cuda_stream) {
+  int st = check_common(B, H, N_txt, N_img, N_ref, d);
+  if (st != JATTN_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || kv_idx == nullptr || kv_cnt == nullptr)
+    return JATTN_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(kv_idx) & 3u) ||
+      (reinterpret_cast<uintptr_t>(kv_cnt) & 3u))
+    return JATTN_ERR_MISALIGNED;
+  AttnProblem pr;
+  std::memset(&pr, 0, sizeof(pr));
+  pr.q = q; pr.k = k; pr.v = v; pr.o = o; pr.lse = lse;
+  pr.B = B; pr.H = H; pr.N = N_txt + N_img + N_ref;
+  pr.softmax_scale = softmax_scale;
+  pr.timeout_ns = kDefaultTimeoutNs;
+  return map_err(launch_attn_bf16_sparse(pr, kv_idx, kv_cnt, static_cast<cudaStream_t>(cuda_stream)));
 }
 
 int jattn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,

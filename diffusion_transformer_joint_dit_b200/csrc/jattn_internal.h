@@ -89,6 +89,22 @@ struct RepairProblem {
 cudaError_t launch_repair_select(const PrologueArgs& a, const RepairProblem& r, cudaStream_t s);
 cudaError_t launch_repair_apply(const RepairProblem& r, int B, int H, int N, float softmax_scale, cudaStream_t s);
 
+// Block-sparse attention (sparse.cu, attn_bf16.cu).
+struct SparseProblem {
+  const void* q;      // bf16 Q' [B, N, H, d]
+  const void* k;      // bf16 K'
+  float* qbar;        // [B, H, n_qb, d] query-block means
+  float* kbar;        // [B, H, n_kb, d] key-block means
+  float* probs;       // nullable [B, H, n_qb, n_kb]
+  int* kv_idx;        // [B, H, n_qb, n_kb]
+  int* kv_cnt;        // [B, H, n_qb]
+  int B, H, N;
+  float softmax_scale, tau;
+};
+
+cudaError_t launch_sparse_select(const SparseProblem& sp, cudaStream_t s);
+cudaError_t launch_attn_bf16_sparse(const AttnProblem& p, const int* kv_idx, const int* kv_cnt, cudaStream_t s);
+
 cudaError_t launch_attn_bf16(const AttnProblem& p, cudaStream_t s);
 cudaError_t launch_attn_fp8(const AttnProblem& p, cudaStream_t s);
 cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t s);

@@ -276,6 +276,61 @@ JATTN_API int jattn_fp8_repair_apply(const void* q8, const float* q_scale, const
                            int B, int H, int N_txt, int N_img, int N_ref, int d, float softmax_scale,
                            void* cuda_stream);
 
+/* Block-sparse attention: query blocks of 256 tokens, key blocks of 128,
+ * counted from token 0 of each (b, h); n_qb = ceil(N / 256),
+ * n_kb = ceil(N / 128). */
+#define JATTN_SPARSE_QBLOCK 256
+#define JATTN_SPARSE_KBLOCK 128
+
+/*
+ * jattn_sparse_select — choose the key blocks each query block attends to.
+ *
+ * Source: Sol-Attention ("Quantized and sparse attention" section of the
+ * tutorial), a generic block-sparse attention whose sparsity a parameter
+ * tau sets (tau = 1.0 in the tutorial; a higher tau is sparser).  The pages
+ * do not define tau; the rule implemented is this reading:
+ *   qbar_i = mean of Q' over query block i, kbar_j = mean of K' over key
+ *   block j (the last blocks partial); p_ij = softmax_j(scale qbar_i.kbar_j);
+ *   key block j is kept for query block i iff p_ij >= tau / n_kb (fp32, the
+ *   threshold one correctly rounded division), and the first j with the
+ *   largest p_ij is always kept.  tau = 0 keeps every block.
+ *
+ * q, k    : bf16 Q', K' [B, N, H, d] (after jattn_prologue).
+ * qbar    : fp32 [B, H, n_qb, d] output (workspace: the query-block means).
+ * kbar    : fp32 [B, H, n_kb, d] output (the key-block means).
+ * probs   : optional fp32 [B, H, n_qb, n_kb] output p_ij; NULL skips it.
+ * kv_idx  : int32 [B, H, n_qb, n_kb] output; row (b, h, i) starts with the
+ *           kept key blocks in increasing order (the rest is not written).
+ * kv_cnt  : int32 [B, H, n_qb] output, the number kept (>= 1).
+ * d == 128; softmax_scale finite > 0; tau finite >= 0; N <= 2^22.
+ * q, k, qbar, kbar 16-byte aligned; probs, kv_idx, kv_cnt 4-byte aligned.
+ */
+JATTN_API int jattn_sparse_select(const void* q, const void* k, float* qbar, float* kbar, float* probs,
+                        int* kv_idx, int* kv_cnt,
+                        int B, int H, int N_txt, int N_img, int N_ref, int d,
+                        float softmax_scale, float tau, void* cuda_stream);
+
+/*
+ * jattn_fwd_bf16_sparse — block-sparse joint attention, BF16 operands.
+ *
+ * Source: the generic block-sparse attention kernel Sol-Attention runs on
+ * ("Quantized and sparse attention" section of the tutorial).
+ *
+ * As jattn_fwd_bf16, except that every query of query block i of (b, h)
+ * attends only to the keys of the key blocks listed in kv_idx[b, h, i, 0 ..
+ * kv_cnt[b, h, i] - 1] (jattn_sparse_select's layout): O = softmax over
+ * those keys of scale * q.k, times their V rows; lse over the same keys.
+ * A query block with count 0 gets O = 0 and lse = -inf.
+ * The list must be strictly increasing key-block indices in [0, n_kb);
+ * counts are clamped to [0, n_kb] and indices into [0, n_kb) so that any
+ * list stays within the tensors, but a list that breaks the rule gives
+ * undefined values.
+ */
+JATTN_API int jattn_fwd_bf16_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const int* kv_idx, const int* kv_cnt,
+                          int B, int H, int N_txt, int N_img, int N_ref, int d,
+                          float softmax_scale, void* cuda_stream);
+
 /* Human-readable name of a jattn_status value (static string, never NULL). */
 JATTN_API const char* jattn_status_string(int status);
 

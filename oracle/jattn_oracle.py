@@ -476,14 +476,16 @@ def block_sparse_attention(q, k, v, keep, scale: float, rows=None,
     key_block = np.arange(N) // kblock
     for b in range(B):
         for h in range(H):
-            for r, t in enumerate(idx):
-                cols = np.nonzero(keep[b, h, t // qblock][key_block])[0]
+            # Rows sharing a query block share the key set.
+            for i in np.unique(idx // qblock):
+                sel = np.nonzero(idx // qblock == i)[0]
+                cols = np.nonzero(keep[b, h, i][key_block])[0]
                 if cols.size == 0:
                     continue
-                s = sc * (f64(k[b, cols, h, :]) @ f64(q[b, t, h, :]))
-                m = np.max(s)
+                s = sc * (f64(q[b, idx[sel], h, :]) @ f64(k[b, cols, h, :]).T)   # [rows, keys]
+                m = np.max(s, axis=1, keepdims=True)
                 p = np.exp(s - m)
-                l = np.sum(p)
-                out[b, r, h, :] = (p / l) @ f64(v[b, cols, h, :])
-                lse[b, h, r] = m + np.log(l)
+                l = np.sum(p, axis=1, keepdims=True)
+                out[b, sel, h, :] = (p / l) @ f64(v[b, cols, h, :])
+                lse[b, h, sel] = (m + np.log(l))[:, 0]
     return out, lse

@@ -156,6 +156,47 @@ def test_rope_table_rejects_bad_arguments(lib):
     assert call(params=J.make_prologue_params(16, 16, rope_theta=-1.0)) == J.JATTN_ERR_INVALID_ARG
 
 
+def test_sparse_select_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(q=A, k=A, qbar=A, kbar=A, probs=None, idx=A, cnt=A, d=128, scale=0.088, tau=1.0, n_img=256)
+        a.update(kw)
+        return J.jattn_sparse_select(a["q"], a["k"], a["qbar"], a["kbar"], a["probs"], a["idx"], a["cnt"], 1, 2,
+                                     32, a["n_img"], 0, a["d"], a["scale"], a["tau"], stream=0, check=False)
+    assert call(d=64) == J.JATTN_ERR_UNSUPPORTED
+    assert call(k=None) == J.JATTN_ERR_INVALID_ARG
+    assert call(qbar=None) == J.JATTN_ERR_INVALID_ARG
+    assert call(cnt=None) == J.JATTN_ERR_INVALID_ARG
+    assert call(tau=-0.5) == J.JATTN_ERR_INVALID_ARG
+    assert call(tau=float("nan")) == J.JATTN_ERR_INVALID_ARG
+    assert call(scale=0.0) == J.JATTN_ERR_INVALID_ARG
+    assert call(n_img=1 << 22) == J.JATTN_ERR_INVALID_ARG            # beyond 2^22 tokens
+    assert call(kbar=MIS) == J.JATTN_ERR_MISALIGNED
+    assert call(probs=A + 2) == J.JATTN_ERR_MISALIGNED
+    assert call(idx=A + 1) == J.JATTN_ERR_MISALIGNED
+
+
+def test_fwd_bf16_sparse_rejects_bad_arguments(lib):
+    def call(**kw):
+        a = dict(q=A, v=A, o=A + 4096, lse=None, idx=A, cnt=A, d=128, scale=0.088)
+        a.update(kw)
+        return J.jattn_fwd_bf16_sparse(a["q"], A, a["v"], a["o"], a["lse"], a["idx"], a["cnt"], 1, 2, 32, 256, 0,
+                                       a["d"], a["scale"], stream=0, check=False)
+    assert call(d=256) == J.JATTN_ERR_UNSUPPORTED
+    assert call(idx=None) == J.JATTN_ERR_INVALID_ARG
+    assert call(cnt=None) == J.JATTN_ERR_INVALID_ARG
+    assert call(o=None) == J.JATTN_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == J.JATTN_ERR_INVALID_ARG
+    assert call(v=MIS) == J.JATTN_ERR_MISALIGNED
+    assert call(cnt=A + 2) == J.JATTN_ERR_MISALIGNED
+    assert call(lse=A + 1) == J.JATTN_ERR_MISALIGNED
+
+
+def test_sparse_block_counts():
+    assert J.sparse_blocks(16896) == (66, 132)
+    assert J.sparse_blocks(300) == (2, 3)
+    assert J.sparse_blocks(1) == (1, 1)
+
+
 def test_selftest_rejects_bad_timeout(lib):
     assert J.jattn_selftest_wait_timeout(0, stream=0, check=False) == J.JATTN_ERR_INVALID_ARG
     assert J.jattn_selftest_wait_timeout(2 * 10 ** 9, stream=0, check=False) == J.JATTN_ERR_INVALID_ARG
