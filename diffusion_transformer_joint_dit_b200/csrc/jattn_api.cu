@@ -461,6 +461,7 @@ int jattn_fp8_repair_apply(const void* q8, const float* q_scale, const void* k8,
   r.q8 = q8; r.q_scale = q_scale; r.k8 = k8; r.v8 = v8; r.k_scale = k_scale; r.v_scale = v_scale;
   r.idx = const_cast<int*>(idx); r.k_sel = const_cast<void*>(k_sel); r.v_sel = const_cast<void*>(v_sel);
   r.o = o; r.lse = lse; r.m = m;
+  r.timeout_ns = kDefaultTimeoutNs;
   return map_err(launch_repair_apply(r, B, H, N, softmax_scale, static_cast<cudaStream_t>(cuda_stream)));
 }
 

@@ -84,6 +84,7 @@ struct RepairProblem {
   void* o;            // bf16 [B, N, H, d], corrected in place
   float* lse;         // [B, H, N], corrected in place
   int m;
+  uint64_t timeout_ns;  // bound of each barrier wait (apply)
 };
 
 cudaError_t launch_repair_select(const PrologueArgs& a, const RepairProblem& r, cudaStream_t s);

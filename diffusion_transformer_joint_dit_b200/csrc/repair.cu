@@ -17,9 +17,9 @@
 //   a = sum_T exp(s_x - L) v_x - exp(s_q - L) v_q,  z = sum_T exp(s_x - L) - exp(s_q - L)
 //   O' = (O + a) / (1 + z),  L' = L + ln(1 + z)
 // with s_x = scale * qd . k'_t and s_q = scale * qd . kd_t.  The products run
-// on the tensor cores (mma.sync m16n8k16, FP16 operands: E4M3 codes and the
-// bf16 rows are exact in FP16 over the range they take, fp32 accumulate);
-// the budget is small (85 keys at N = 16896), so this pass is short.
+// on the tensor cores (tcgen05, TMEM accumulators; E4M3 codes and the bf16
+// rows are exact in FP16 over the range they take); the budget is small (85
+// keys at N = 16896), so this pass is short.
 #include "jattn_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -214,26 +214,45 @@ repair_gather_kernel(const __grid_constant__ PrologueArgs a, const int* __restri
 }
 
 // ----------------------------------------------------------- 4. apply ----
-// CTA = 8 warps x 16 query rows = 128 query rows (two FP8 scale blocks) per
-// pass.  The selected keys are staged in shared memory as FP16, up to
-// kStageMax at a time: when they all fit, a CTA stages them once and walks a
-// run of passes (about one CTA per SM over the grid); otherwise each CTA
-// takes one pass and restages per group of kStageMax keys.
-constexpr int kApplyWarps = 8;
-constexpr int kApplyQ = kApplyWarps * 16;  // query rows per pass
-constexpr int kStageMax = 128;             // selected keys staged at a time
-constexpr int kKStride = kD + 8;         // fp16 per K row (bank-conflict padding)
-constexpr int kVStride = kStageMax + 8;  // fp16 per transposed V row
+// tcgen05 correction pass.  CTA = 4 warps; a pass covers 128 query rows, one
+// per thread and TMEM lane.  The selected keys of the (b, h) (up to
+// kStageMax per group, padded to P, a multiple of 32) sit in shared memory
+// in the 128-byte-swizzled layouts the MMAs read:
+//   Kx16  exact K' as FP16, K-major (two 64-channel boxes of P rows)
+//   Kq8   K codes (E4M3), K-major (one box of P rows)
+//   V16   [exact V ; V codes] as FP16, MN-major (two 64-channel boxes of 2P rows)
+// Per pass the Q codes land twice, as an E4M3 tile and widened to FP16, and
+// one thread issues
+//   S_x = Q16 . Kx16^T  (kind::f16)                 -> TMEM [0, P)
+//   S_q = Q8  . Kq8^T   (kind::f8f6f4)              -> TMEM [128, 128 + P)
+// each thread turns its row into W = [w_x | -w_q s_v] (FP16 pairs, TMEM
+// [384, 384 + P)) and z, and then
+//   O_c = W . V16       (kind::f16, A from TMEM)    -> TMEM [256, 384)
+// after which the thread rewrites its O and L rows.  With more than
+// kStageMax selected keys, the groups run one after another inside a pass,
+// accumulating O_c and z.  Exact K' and V rows must lie within the FP16
+// range (E4M3 codes and bf16 rows of moderate size are exact in FP16).
+constexpr int kApplyThreads = 128;
+constexpr int kApplyQ = 128;            // query rows per pass (= TMEM lanes)
+constexpr int kStageMax = 128;          // selected keys per group
+constexpr uint32_t kColSx = 0, kColSq = 128, kColO = 256, kColW = 384;
+constexpr uint32_t kApplyTmemCols = 512;
 
-struct ApplySmem {
-  uint8_t q[kApplyQ][kD];                // Q codes of the current query block
-  __half kx[kStageMax][kKStride];        // exact K' (fp16)
-  __half kq[kStageMax][kKStride];        // K codes (fp16)
-  __half vx[kD][kVStride];               // exact V, transposed
-  __half vq[kD][kVStride];               // V codes, transposed
-  float ks[kStageMax], vs[kStageMax];
+struct ApplyCtrl {
+  uint64_t s_full;
+  uint64_t o_full;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
 };
-constexpr int kApplySmemBytes = static_cast<int>(sizeof(ApplySmem)) + 128;
+
+constexpr int kSmQ8 = 0;                              // 128 rows x 128 B
+constexpr int kSmQ16 = kSmQ8 + kApplyQ * 128;         // 2 boxes x 128 rows x 128 B
+constexpr int kSmKx = kSmQ16 + 2 * kApplyQ * 128;     // 2 boxes x P rows x 128 B
+constexpr int kSmKq = kSmKx + 2 * kStageMax * 128;    // P rows x 128 B
+constexpr int kSmV = kSmKq + kStageMax * 128;         // 2 boxes x 2P rows x 128 B
+constexpr int kSmCtrl = kSmV + 4 * kStageMax * 128;
+constexpr int kApplySmemBytes = kSmCtrl + static_cast<int>(sizeof(ApplyCtrl)) + 1024;
 
 struct ApplyParams {
   const uint8_t* q8;
@@ -250,198 +269,292 @@ struct ApplyParams {
   int H, N, m;
   int passes_per_cta;
   float scale_log2;
+  uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// Byte offset of 16-byte chunk `chunk` of row `r` in a 128-byte-swizzled
+// tile (rows of 128 B, 1024-byte aligned base).
+__device__ __forceinline__ uint32_t sw128(int r, int chunk) {
+  return static_cast<uint32_t>(r * 128 + ((chunk ^ (r & 7)) << 4));
 }
 
-__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
+// 8 bf16 -> 8 FP16 (exact for moderate magnitudes).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  return make_uint4(bf16x2_to_f16x2(v.x), bf16x2_to_f16x2(v.y), bf16x2_to_f16x2(v.z), bf16x2_to_f16x2(v.w));
 }
 
-// Stage selected keys [i0, i0 + n) of (b, h) into shared memory (FP16),
-// zero-padding up to a multiple of 32.
-__device__ __forceinline__ void stage_keys(const ApplyParams& p, ApplySmem& sm, int b, int h, size_t bh, int nblk,
-                                           int i0, int n) {
-  const int n32 = (n + 31) & ~31;
-  for (int e = threadIdx.x; e < n32 * (kD / 8); e += blockDim.x) {
-    const int i = e / (kD / 8), c8 = (e % (kD / 8)) * 8;
+// 16 E4M3 codes -> 16 FP16 values (exact), as two 16-byte chunks.
+__device__ __forceinline__ void e4m3x16_to_f16(uint4 c, uint4& lo, uint4& hi) {
+  lo = make_uint4(e4m3x2_to_f16x2(c.x), e4m3x2_to_f16x2(c.x >> 16), e4m3x2_to_f16x2(c.y),
+                  e4m3x2_to_f16x2(c.y >> 16));
+  hi = make_uint4(e4m3x2_to_f16x2(c.z), e4m3x2_to_f16x2(c.z >> 16), e4m3x2_to_f16x2(c.w),
+                  e4m3x2_to_f16x2(c.w >> 16));
+}
+
+// Stage selected keys [i0, i0 + ns) of (b, h), zero-padded to P rows.
+__device__ __forceinline__ void apply_stage_keys(const ApplyParams& p, uint8_t* sm, float* s_ks, float* s_vs, int b,
+                                                 int h, size_t bh, int nblk, int i0, int ns, int P) {
+#pragma unroll 4
+  for (int e = threadIdx.x; e < P * 16; e += kApplyThreads) {  // exact rows: 8 channels per task
+    const int i = e >> 4, c8 = e & 15;
     uint4 kx = make_uint4(0, 0, 0, 0), vx = kx;
-    uint2 kc = make_uint2(0, 0), vc = kc;
-    if (i < n) {
-      const size_t sr = (bh * p.m + i0 + i) * kD + c8;
+    if (i < ns) {
+      const size_t sr = (bh * p.m + i0 + i) * kD + c8 * 8;
       kx = __ldg(reinterpret_cast<const uint4*>(p.k_sel + sr));
       vx = __ldg(reinterpret_cast<const uint4*>(p.v_sel + sr));
-      const int t = __ldg(p.idx + bh * p.m + i0 + i);
-      const size_t cr = ((static_cast<size_t>(b) * p.N + t) * p.H + h) * kD + c8;
-      kc = __ldg(reinterpret_cast<const uint2*>(p.k8 + cr));
-      vc = __ldg(reinterpret_cast<const uint2*>(p.v8 + cr));
-      if (c8 == 0) {
-        sm.ks[i] = __ldg(p.k_scale + bh * nblk + t / kQuantBlock);
-        sm.vs[i] = __ldg(p.v_scale + bh * nblk + t / kQuantBlock);
-      }
-    } else if (c8 == 0) {
-      sm.ks[i] = 0.f;
-      sm.vs[i] = 0.f;
     }
-    const uint32_t kxw[4] = {kx.x, kx.y, kx.z, kx.w}, vxw[4] = {vx.x, vx.y, vx.z, vx.w};
-    const uint32_t kcw[2] = {kc.x, kc.y}, vcw[2] = {vc.x, vc.y};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      *reinterpret_cast<uint32_t*>(&sm.kx[i][c8 + 2 * j]) = bf16x2_to_f16x2(kxw[j]);
-      *reinterpret_cast<uint32_t*>(&sm.kq[i][c8 + 2 * j]) = e4m3x2_to_f16x2(kcw[j >> 1] >> (16 * (j & 1)));
-      const uint32_t v2 = bf16x2_to_f16x2(vxw[j]);
-      const uint32_t vq2 = e4m3x2_to_f16x2(vcw[j >> 1] >> (16 * (j & 1)));
-      sm.vx[c8 + 2 * j][i] = *reinterpret_cast<const __half*>(&v2);
-      sm.vx[c8 + 2 * j + 1][i] = *(reinterpret_cast<const __half*>(&v2) + 1);
-      sm.vq[c8 + 2 * j][i] = *reinterpret_cast<const __half*>(&vq2);
-      sm.vq[c8 + 2 * j + 1][i] = *(reinterpret_cast<const __half*>(&vq2) + 1);
+    const int box = c8 >> 3, ch = c8 & 7;
+    *reinterpret_cast<uint4*>(sm + kSmKx + box * P * 128 + sw128(i, ch)) = bf16x8_to_f16x8(kx);
+    *reinterpret_cast<uint4*>(sm + kSmV + box * 2 * P * 128 + sw128(i, ch)) = bf16x8_to_f16x8(vx);
+  }
+#pragma unroll 3
+  for (int e = threadIdx.x; e < P * 8; e += kApplyThreads) {   // codes: 16 channels per task
+    const int i = e >> 3, c16 = e & 7;
+    uint4 kc = make_uint4(0, 0, 0, 0), vc = kc;
+    float ksc = 0.f, vsc = 0.f;
+    if (i < ns) {
+      const int t = min(max(__ldg(p.idx + bh * p.m + i0 + i), 0), p.N - 1);  // in range for any list
+      const size_t cr = ((static_cast<size_t>(b) * p.N + t) * p.H + h) * kD + c16 * 16;
+      kc = __ldg(reinterpret_cast<const uint4*>(p.k8 + cr));
+      vc = __ldg(reinterpret_cast<const uint4*>(p.v8 + cr));
+      ksc = __ldg(p.k_scale + bh * nblk + t / kQuantBlock);
+      vsc = __ldg(p.v_scale + bh * nblk + t / kQuantBlock);
+    }
+    *reinterpret_cast<uint4*>(sm + kSmKq + sw128(i, c16)) = kc;
+    uint4 lo, hi;
+    e4m3x16_to_f16(vc, lo, hi);
+    uint8_t* vbox = sm + kSmV + (c16 >> 2) * 2 * P * 128;
+    const int c8 = (c16 & 3) * 2;
+    *reinterpret_cast<uint4*>(vbox + sw128(P + i, c8)) = lo;
+    *reinterpret_cast<uint4*>(vbox + sw128(P + i, c8 + 1)) = hi;
+    if (c16 == 0) {
+      s_ks[i] = ksc;
+      s_vs[i] = vsc;
     }
   }
 }
 
-__global__ void __launch_bounds__(kApplyWarps * 32, 1)
+// This thread's 8 chunks of the pass's Q codes (zero past N): task e =
+// thread + 128 k, row e / 8, chunk e % 8.
+__device__ __forceinline__ void apply_load_q(const ApplyParams& p, int b, int h, int q0, uint4 (&qn)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int e = threadIdx.x + k * kApplyThreads;
+    const int row = q0 + (e >> 3);
+    qn[k] = make_uint4(0, 0, 0, 0);
+    if (row < p.N)
+      qn[k] = __ldg(reinterpret_cast<const uint4*>(p.q8 + ((static_cast<size_t>(b) * p.N + row) * p.H + h) * kD) +
+                    (e & 7));
+  }
+}
+
+__device__ __forceinline__ void apply_store_q(uint8_t* sm, const uint4 (&qn)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int e = threadIdx.x + k * kApplyThreads;
+    const int r = e >> 3, c16 = e & 7;
+    *reinterpret_cast<uint4*>(sm + kSmQ8 + sw128(r, c16)) = qn[k];
+    uint4 lo, hi;
+    e4m3x16_to_f16(qn[k], lo, hi);
+    uint8_t* qbox = sm + kSmQ16 + (c16 >> 2) * kApplyQ * 128;
+    const int c8 = (c16 & 3) * 2;
+    *reinterpret_cast<uint4*>(qbox + sw128(r, c8)) = lo;
+    *reinterpret_cast<uint4*>(qbox + sw128(r, c8 + 1)) = hi;
+  }
+}
+
+__global__ void __launch_bounds__(kApplyThreads, 1)
 repair_apply_kernel(const __grid_constant__ ApplyParams p) {
   extern __shared__ uint8_t smem_raw[];
-  ApplySmem& sm = *reinterpret_cast<ApplySmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, tq = lane & 3;
+  __shared__ float s_ks[kStageMax], s_vs[kStageMax];  // block scales of the staged keys
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  ApplyCtrl* ctrl = reinterpret_cast<ApplyCtrl*>(sm + kSmCtrl);
+  volatile int* abort_flag = &ctrl->abort;
+  const int warp = threadIdx.x >> 5;
   const int h = blockIdx.y, b = blockIdx.z;
-  const int N = p.N, H = p.H, m = p.m;
+  const int N = p.N, m = p.m;
   const int nblk = (N + kQuantBlock - 1) / kQuantBlock;
-  const size_t bh = static_cast<size_t>(b) * H + h;
-  const bool staged_once = m <= kStageMax;
+  const size_t bh = static_cast<size_t>(b) * p.H + h;
+  const int ngroups = (m + kStageMax - 1) / kStageMax;
   const int npass = (N + kApplyQ - 1) / kApplyQ;
-  const int qb0 = blockIdx.x * p.passes_per_cta;
-  const int qb1 = min(qb0 + p.passes_per_cta, npass);
+  const int pass0 = blockIdx.x * p.passes_per_cta;
+  const int pass1 = min(pass0 + p.passes_per_cta, npass);
   const float log2e = 1.4426950408889634f;
 
-  if (staged_once) {
-    stage_keys(p, sm, b, h, bh, nblk, 0, m);
-    __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->s_full, 1);
+    mbar_init(&ctrl->o_full, 1);
+    mbar_init(&ctrl->mma_done, 1);
+    ctrl->abort = 0;
+    fence_barrier_init();
   }
-#pragma unroll 1
-  for (int qb = qb0; qb < qb1; ++qb) {
-    const int q0 = qb * kApplyQ;
-    __syncthreads();  // previous block's readers of sm.q are done
-    for (int e = threadIdx.x; e < kApplyQ * (kD / 16); e += blockDim.x) {
-      const int rr = e / (kD / 16), cc = e % (kD / 16);
-      const int q = q0 + rr;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (q < N) v = __ldg(reinterpret_cast<const uint4*>(p.q8 + ((static_cast<size_t>(b) * N + q) * H + h) * kD) + cc);
-      *reinterpret_cast<uint4*>(&sm.q[rr][cc * 16]) = v;
-    }
-    __syncthreads();
-    // A fragments (this warp's 16 query rows x 128 channels), FP16 codes.
-    uint32_t qa[kD / 16][4];
-    {
-      const int ra = warp * 16 + g, rb = ra + 8;
-#pragma unroll
-      for (int ks = 0; ks < kD / 16; ++ks) {
-        const int c0 = ks * 16 + 2 * tq;
-        qa[ks][0] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&sm.q[ra][c0]));
-        qa[ks][1] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&sm.q[rb][c0]));
-        qa[ks][2] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&sm.q[ra][c0 + 8]));
-        qa[ks][3] = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(&sm.q[rb][c0 + 8]));
-      }
-    }
-    const float qsc = __ldg(p.q_scale + bh * nblk + (q0 + warp * 16) / kQuantBlock);
-    const int row_a = q0 + warp * 16 + g, row_b = row_a + 8;
-    const float l2a = row_a < N ? p.lse[bh * N + row_a] * log2e : 0.f;
-    const float l2b = row_b < N ? p.lse[bh * N + row_b] * log2e : 0.f;
-    const float sx = qsc * p.scale_log2;
-    float acc[kD / 8][4];
-#pragma unroll
-    for (int n = 0; n < kD / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    float za = 0.f, zb = 0.f;  // sum exp(s_x - L) - exp(s_q - L), rows a, b
+  if (warp == 0) {
+    tmem_alloc(&ctrl->tmem_base, kApplyTmemCols);
+    tmem_relinquish();
+  }
+  if (ngroups == 1) {
+    apply_stage_keys(p, sm, s_ks, s_vs, b, h, bh, nblk, 0, m, (m + 31) & ~31);
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  const uint32_t lane_sel = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t idesc_pv = make_idesc(0, 0, true, kApplyQ, kD);  // f16 W (TMEM) x f16 V (MN-major)
+  uint32_t s_phase = 0, o_phase = 0;
+  bool ok = true;
 
+  // Per-pass inputs of this thread's row, loaded one pass ahead: the Q
+  // codes, the row's Q scale and its log-sum-exp.
+  uint4 qn[8];
+  float qsc_n = 0.f, lse_n = 0.f;
+  auto prefetch = [&](int q0) {
+    apply_load_q(p, b, h, q0, qn);
+    const int r = q0 + static_cast<int>(threadIdx.x);
+    qsc_n = r < N ? __ldg(p.q_scale + bh * nblk + r / kQuantBlock) : 0.f;
+    lse_n = r < N ? p.lse[bh * N + r] : 0.f;
+  };
+  if (pass0 < pass1) prefetch(pass0 * kApplyQ);
 #pragma unroll 1
-    for (int s0 = 0; s0 < m; s0 += kStageMax) {
-      const int ns = min(kStageMax, m - s0);
-      if (!staged_once) {
-        __syncthreads();
-        stage_keys(p, sm, b, h, bh, nblk, s0, ns);
-        __syncthreads();
-      }
+  for (int pass = pass0; pass < pass1; ++pass) {
+    const int q0 = pass * kApplyQ;
+    apply_store_q(sm, qn);
+    fence_proxy_async_smem();
+    const int row = q0 + threadIdx.x;
+    const bool live = row < N;
+    const float lse_row = lse_n;
+    const float l2 = lse_row * log2e;
+    const float sx = qsc_n * p.scale_log2;
+    float z = 0.f;  // sum over selected keys of exp(s_x - L) - exp(s_q - L)
+    __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * N + (live ? row : 0)) * p.H + h) * kD;
+    uint4 o_in[kD / 8];
 #pragma unroll 1
-      for (int c0k = 0; c0k < ns; c0k += 32) {
-        uint32_t wa[4][4];  // A fragments of [w_x (32 keys) | -w_q (32 keys)]
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          float cx[4] = {0.f, 0.f, 0.f, 0.f}, cq[4] = {0.f, 0.f, 0.f, 0.f};
-          const int key = c0k + nt * 8 + g;  // B column of this lane
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const int cc = ks * 16 + 2 * tq;
-            mma16816(cx, qa[ks], *reinterpret_cast<const uint32_t*>(&sm.kx[key][cc]),
-                     *reinterpret_cast<const uint32_t*>(&sm.kx[key][cc + 8]));
-            mma16816(cq, qa[ks], *reinterpret_cast<const uint32_t*>(&sm.kq[key][cc]),
-                     *reinterpret_cast<const uint32_t*>(&sm.kq[key][cc + 8]));
-          }
-          float wx[4], wq[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int kk = c0k + nt * 8 + 2 * tq + (j & 1);
-            const bool live = kk < ns;
-            const float l2 = j < 2 ? l2a : l2b;
-            wx[j] = live ? ex2_approx(cx[j] * sx - l2) : 0.f;
-            wq[j] = live ? ex2_approx(cq[j] * (sx * sm.ks[kk]) - l2) : 0.f;
-            if (j < 2) za += wx[j] - wq[j]; else zb += wx[j] - wq[j];
-            wq[j] *= sm.vs[kk];  // V's block scale folded into the weight
-          }
-          const int kstep = nt >> 1, hi = nt & 1;
-          wa[kstep][2 * hi] = pack_h2(wx[0], wx[1]);
-          wa[kstep][2 * hi + 1] = pack_h2(wx[2], wx[3]);
-          wa[2 + kstep][2 * hi] = pack_h2(-wq[0], -wq[1]);
-          wa[2 + kstep][2 * hi + 1] = pack_h2(-wq[2], -wq[3]);
-        }
-        // acc += [w_x | -w_q] [V_x ; V_q]
-#pragma unroll
-        for (int n = 0; n < kD / 8; ++n) {
-          const int dcol = n * 8 + g;
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const __half(*vt)[kVStride] = k4 < 2 ? sm.vx : sm.vq;
-            const int kb = c0k + (k4 & 1) * 16 + 2 * tq;
-            mma16816(acc[n], wa[k4], *reinterpret_cast<const uint32_t*>(&vt[dcol][kb]),
-                     *reinterpret_cast<const uint32_t*>(&vt[dcol][kb + 8]));
-          }
-        }
+    for (int g = 0; g < ngroups; ++g) {
+      const int ns = min(kStageMax, m - g * kStageMax);
+      const int P = (ns + 31) & ~31;
+      if (ngroups > 1) {
+        // The previous group's MMAs have completed (o_full waited below).
+        apply_stage_keys(p, sm, s_ks, s_vs, b, h, bh, nblk, g * kStageMax, ns, P);
+        fence_proxy_async_smem();
       }
+      __syncthreads();  // Q (and keys) written; previous readers of TMEM done
+      if (threadIdx.x == 0 && ok) {
+        tc_fence_after();
+        const uint32_t idesc_x = make_idesc(0, 0, false, kApplyQ, P);  // f16 x f16, K-major
+        const uint32_t idesc_q = make_idesc(0, 0, false, kApplyQ, P);  // e4m3 x e4m3, K-major
+        const uint32_t q16 = smem_u32(sm + kSmQ16), kx = smem_u32(sm + kSmKx);
+        const uint32_t q8 = smem_u32(sm + kSmQ8), kq = smem_u32(sm + kSmKq);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (kApplyQ * 128) + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * (P * 128) + (kk & 3) * 32;
+          mma_f16_ss(tmem + kColSx, smem_desc_sw128(q16 + aoff, 16, 1024), smem_desc_sw128(kx + boff, 16, 1024),
+                     idesc_x, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < kD / 32; ++kk)
+          mma_f8_ss(tmem + kColSq, smem_desc_sw128(q8 + kk * 32, 16, 1024), smem_desc_sw128(kq + kk * 32, 16, 1024),
+                    idesc_q, kk > 0 ? 1u : 0u);
+        mma_commit(&ctrl->s_full);
+      }
+      if (g == 0 && pass + 1 < pass1) prefetch(q0 + kApplyQ);  // next pass, in flight meanwhile
+      if (ok) ok = mbar_wait(&ctrl->s_full, s_phase & 1u, abort_flag, p.timeout_ns);
+      ++s_phase;
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < P; c0 += 32) {
+          uint32_t ax[32], aq[32];
+          tmem_ld32(tmem + lane_sel + kColSx + c0, ax);
+          tmem_ld32(tmem + lane_sel + kColSq + c0, aq);
+          tmem_ld_wait(ax);
+          tmem_ld_wait(aq);
+          uint32_t wx[16], wq[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float ex[2], eq[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int key = c0 + j + u;
+              const bool in = key < ns;
+              ex[u] = in ? ex2_approx(__uint_as_float(ax[j + u]) * sx - l2) : 0.f;
+              eq[u] = in ? ex2_approx(__uint_as_float(aq[j + u]) * (sx * s_ks[key]) - l2) : 0.f;
+              z += ex[u] - eq[u];
+              eq[u] *= -s_vs[key];  // V's block scale folded into the weight of the codes
+            }
+            wx[j >> 1] = pack_f16x2(ex[0], ex[1]);
+            wq[j >> 1] = pack_f16x2(eq[0], eq[1]);
+          }
+          tmem_st16(tmem + lane_sel + kColW + c0 / 2, wx);
+          tmem_st16(tmem + lane_sel + kColW + P / 2 + c0 / 2, wq);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      __syncthreads();  // W of every row is in TMEM
+      if (threadIdx.x == 0 && ok) {
+        tc_fence_after();
+        const uint32_t v16 = smem_u32(sm + kSmV);
+#pragma unroll 1
+        for (int kk = 0; kk < (2 * P) / 16; ++kk)
+          mma_f16_ts(tmem + kColO, tmem + kColW + kk * 8, smem_desc_sw128(v16 + kk * 16 * 128, 2 * P * 128, 1024),
+                     idesc_pv, (g > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&ctrl->o_full);
+      }
+      if (g == ngroups - 1) {
+        // This row of O, in flight while the tensor core computes O_c.
+#pragma unroll
+        for (int i = 0; i < kD / 8; ++i)
+          o_in[i] = live ? *reinterpret_cast<const uint4*>(orow + i * 8) : make_uint4(0, 0, 0, 0);
+      }
+      if (ok) ok = mbar_wait(&ctrl->o_full, o_phase & 1u, abort_flag, p.timeout_ns);
+      ++o_phase;
+      ok = __all_sync(0xffffffffu, ok);
     }
+    // Epilogue: O' = (O + a) / (1 + z), L' = L + ln(1 + z).
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / (1.f + z);
+#pragma unroll
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t a[32];
+        uint4 ov[4];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) ov[q4] = o_in[c * 4 + q4];
+        tmem_ld32(tmem + lane_sel + kColO + c * 32, a);
+        tmem_ld_wait(a);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t w[4] = {ov[q4].x, ov[q4].y, ov[q4].z, ov[q4].w};
+          uint32_t r[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float lo = (__uint_as_float(w[i] << 16) + __uint_as_float(a[q4 * 8 + 2 * i])) * inv;
+            const float hi = (__uint_as_float(w[i] & 0xFFFF0000u) + __uint_as_float(a[q4 * 8 + 2 * i + 1])) * inv;
+            r[i] = pack_bf16x2(lo, hi);
+          }
+          if (live) *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = make_uint4(r[0], r[1], r[2], r[3]);
+        }
+      }
+      if (live) p.lse[bh * N + row] = lse_row + __logf(1.f + z);
+    }
+    tc_fence_before();
+    __syncthreads();  // O_c read before the next pass's MMAs overwrite TMEM
+  }
 
-    // Row sums over the quad, then O' = (O + a) / (1 + z), L' = L + ln(1 + z).
-    za += __shfl_xor_sync(0xffffffffu, za, 1);
-    za += __shfl_xor_sync(0xffffffffu, za, 2);
-    zb += __shfl_xor_sync(0xffffffffu, zb, 1);
-    zb += __shfl_xor_sync(0xffffffffu, zb, 2);
-    const float ia = 1.f / (1.f + za), ib = 1.f / (1.f + zb);
-#pragma unroll
-    for (int n = 0; n < kD / 8; ++n) {
-      const int c = n * 8 + 2 * tq;
-      if (row_a < N) {
-        __nv_bfloat162* o2 =
-            reinterpret_cast<__nv_bfloat162*>(p.o + ((static_cast<size_t>(b) * N + row_a) * H + h) * kD + c);
-        const float2 f = __bfloat1622float2(*o2);
-        *o2 = __floats2bfloat162_rn((f.x + acc[n][0]) * ia, (f.y + acc[n][1]) * ia);
-      }
-      if (row_b < N) {
-        __nv_bfloat162* o2 =
-            reinterpret_cast<__nv_bfloat162*>(p.o + ((static_cast<size_t>(b) * N + row_b) * H + h) * kD + c);
-        const float2 f = __bfloat1622float2(*o2);
-        *o2 = __floats2bfloat162_rn((f.x + acc[n][2]) * ib, (f.y + acc[n][3]) * ib);
-      }
-    }
-    if (tq == 0) {
-      if (row_a < N) p.lse[bh * N + row_a] += __logf(1.f + za);
-      if (row_b < N) p.lse[bh * N + row_b] += __logf(1.f + zb);
-    }
+  // Teardown: every issued MMA has completed before TMEM is released.
+  if (threadIdx.x == 0) {
+    mma_commit(&ctrl->mma_done);
+    int never = 0;
+    mbar_wait(&ctrl->mma_done, 0, &never, p.timeout_ns);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kApplyTmemCols);
   }
 }
 
@@ -480,16 +593,18 @@ cudaError_t launch_repair_apply(const RepairProblem& r, int B, int H, int N, flo
   p.H = H;
   p.N = N;
   p.m = r.m;
-  // Keys staged once: about one CTA per SM, each walking a run of passes.
+  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
+  p.timeout_ns = r.timeout_ns;
+  // Keys staged once: about one CTA per SM, each walking a run of passes;
+  // more keys than one group: one pass per CTA.
   const int npass = (N + kApplyQ - 1) / kApplyQ;
   int per_head = 1;
   if (r.m <= kStageMax) per_head = std::max(1, std::min(npass, device_sm_count() / std::max(1, B * H)));
   p.passes_per_cta = r.m <= kStageMax ? (npass + per_head - 1) / per_head : 1;
-  p.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
   cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(repair_apply_kernel), kApplySmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((npass + p.passes_per_cta - 1) / p.passes_per_cta, H, B);
-  repair_apply_kernel<<<grid, kApplyWarps * 32, kApplySmemBytes, s>>>(p);
+  repair_apply_kernel<<<grid, kApplyThreads, kApplySmemBytes, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -266,9 +266,14 @@ JATTN_API int jattn_fp8_repair_select(const void* k, const void* v, const void* 
  *          attention in which the selected keys use their exact rows:
  *          with a = sum over them of exp(s_x - L) v_x - exp(s_q - L) v_q and
  *          z the same sum without v, O' = (O + a) / (1 + z), L' = L + ln(1+z),
- *          s_x = scale qd.k'_t and s_q = scale qd.kd_t (tensor-core products
- *          of FP16 operands, fp32 accumulation).
+ *          s_x = scale qd.k'_t and s_q = scale qd.kd_t (tensor-core products,
+ *          fp32 accumulation: s_x from FP16 operands, s_q from the E4M3
+ *          codes).  The exact K' and V rows are used as FP16, so they must
+ *          lie within the FP16 range.
  * m == 0 leaves o and lse unchanged.  softmax_scale as for jattn_fwd_fp8.
+ * Token indices in idx are clamped into [0, N); a list that is not
+ * jattn_fp8_repair_select's gives undefined values, never an access
+ * outside the tensors.
  */
 JATTN_API int jattn_fp8_repair_apply(const void* q8, const float* q_scale, const void* k8, const void* v8,
                            const float* k_scale, const float* v_scale, const int* idx,
