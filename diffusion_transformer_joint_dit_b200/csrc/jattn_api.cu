@@ -152,26 +152,33 @@ int device_sm_count() {
 }
 
 cudaError_t set_smem_attr(const void* func, int bytes) {
+  // Remembers the largest limit set per device and kernel; a kernel whose
+  // shared memory depends on the problem size is raised again when a call
+  // needs more.
   constexpr int kMaxDev = 64;
-  constexpr int kMaxFuncs = 8;
+  constexpr int kMaxFuncs = 16;
   static std::mutex mu;
   static const void* done_func[kMaxDev][kMaxFuncs] = {};
+  static int done_bytes[kMaxDev][kMaxFuncs] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
+  int slot = -1;
   if (dev >= 0 && dev < kMaxDev) {
-    for (int i = 0; i < kMaxFuncs; ++i)
-      if (done_func[dev][i] == func) return cudaSuccess;
+    for (int i = 0; i < kMaxFuncs && slot < 0; ++i)
+      if (done_func[dev][i] == func) slot = i;
+    if (slot >= 0 && done_bytes[dev][slot] >= bytes) return cudaSuccess;
   }
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < kMaxDev) {
-    for (int i = 0; i < kMaxFuncs; ++i)
-      if (done_func[dev][i] == nullptr) {
-        done_func[dev][i] = func;
-        break;
-      }
+    for (int i = 0; i < kMaxFuncs && slot < 0; ++i)
+      if (done_func[dev][i] == nullptr) slot = i;
+    if (slot >= 0) {
+      done_func[dev][slot] = func;
+      done_bytes[dev][slot] = bytes;
+    }
   }
   return cudaSuccess;
 }
