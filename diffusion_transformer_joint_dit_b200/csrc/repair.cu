@@ -107,31 +107,14 @@ repair_error_kernel(const __grid_constant__ PrologueArgs a, const uint8_t* __res
 // One CTA per (b, h).  Errors are >= 0, so their bit patterns order like
 // unsigned integers: four 8-bit radix passes find the m-th largest value
 // theta and how many tokens equal to theta are taken (the first ones in
-// token order); a block-wide scan then lists the selected tokens in order.
+// token order); the warps then list the selected tokens of their token
+// segments in order.
 constexpr int kSelThreads = 512;
-
-__device__ __forceinline__ unsigned block_excl_scan(unsigned flag, unsigned* warp_tot, unsigned& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned bal = __ballot_sync(0xffffffffu, flag != 0u);
-  const unsigned within = __popc(bal & ((1u << lane) - 1u));
-  __syncthreads();
-  if (lane == 0) warp_tot[warp] = __popc(bal);
-  __syncthreads();
-  unsigned before = 0, all = 0;
-  for (int w = 0; w < kSelThreads / 32; ++w) {
-    const unsigned n = warp_tot[w];
-    before += w < warp ? n : 0u;
-    all += n;
-  }
-  total = all;
-  return before + within;
-}
 
 __global__ void __launch_bounds__(kSelThreads)
 repair_select_kernel(const float* __restrict__ err, int N, int m, int* __restrict__ idx) {
   __shared__ unsigned hist[256];
   __shared__ unsigned s_prefix, s_k;
-  __shared__ unsigned warp_tot[kSelThreads / 32];
   const int bh = blockIdx.y * gridDim.x + blockIdx.x;  // (b, h) row of err / idx
   const float* e = err + static_cast<size_t>(bh) * N;
   int* out = idx + static_cast<size_t>(bh) * m;
@@ -145,18 +128,38 @@ repair_select_kernel(const float* __restrict__ err, int N, int m, int* __restric
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      unsigned cum = 0, dsel = 0, kk = k;
-      for (int d = 255; d >= 0; --d) {
-        if (cum + hist[d] >= k) {
-          dsel = static_cast<unsigned>(d);
-          kk = k - cum;
-          break;
-        }
-        cum += hist[d];
+    if (threadIdx.x < 32) {
+      // The digit d with count(digits > d) < k <= count(digits >= d): lane l
+      // holds digits 8 l .. 8 l + 7; suffix sums over the lanes find the
+      // lane that holds d, which then walks its eight counts.
+      const int lane = threadIdx.x;
+      unsigned c[8], tot = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c[i] = hist[lane * 8 + i];
+        tot += c[i];
       }
-      s_prefix = prefix | (dsel << shift);
-      s_k = kk;
+      unsigned incl = tot;  // digits >= 8 lane
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += v;
+      }
+      unsigned cum = incl - tot;  // digits > 8 lane + 7
+      if (cum < k && k <= incl) {
+        unsigned dsel = 0, kk = k;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+          if (cum + c[i] >= k) {
+            dsel = static_cast<unsigned>(lane * 8 + i);
+            kk = k - cum;
+            break;
+          }
+          cum += c[i];
+        }
+        s_prefix = prefix | (dsel << shift);
+        s_k = kk;
+      }
     }
     __syncthreads();
     prefix = s_prefix;
@@ -164,20 +167,44 @@ repair_select_kernel(const float* __restrict__ err, int N, int m, int* __restric
     mask |= 255u << shift;
   }
   const unsigned theta = prefix, take_eq = k;  // m-th largest value; ties of it to take
-  unsigned eq_seen = 0, written = 0;
-  for (int t0 = 0; t0 < N; t0 += kSelThreads) {
-    const int t = t0 + threadIdx.x;
-    const unsigned u = t < N ? __float_as_uint(__ldg(e + t)) : 0u;
-    const bool gt = t < N && u > theta;
-    const bool eq = t < N && u == theta;
-    unsigned eq_total;
-    const unsigned eq_rank = block_excl_scan(eq ? 1u : 0u, warp_tot, eq_total);
-    const bool sel = gt || (eq && eq_seen + eq_rank < take_eq);
-    unsigned sel_total;
-    const unsigned pos = block_excl_scan(sel ? 1u : 0u, warp_tot, sel_total);
-    if (sel) out[written + pos] = t;
-    eq_seen += eq_total;
-    written += sel_total;
+  // Listing: warp w owns the contiguous token segment [w seg, (w + 1) seg).
+  // One counting sweep, one barrier for the per-warp counts, then each warp
+  // writes its selected tokens in order with ballots.
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = kSelThreads / 32;
+  __shared__ unsigned s_gt[kWarps], s_eq[kWarps];
+  const int seg = (N + kWarps - 1) / kWarps;
+  const int s0 = min(N, warp * seg), s1 = min(N, s0 + seg);
+  unsigned n_gt = 0, n_eq = 0;
+  for (int base = s0; base < s1; base += 32) {
+    const int t = base + lane;
+    const unsigned u = t < s1 ? __float_as_uint(__ldg(e + t)) : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, t < s1 && u > theta));
+    n_eq += __popc(__ballot_sync(0xffffffffu, t < s1 && u == theta));
+  }
+  if (lane == 0) {
+    s_gt[warp] = n_gt;
+    s_eq[warp] = n_eq;
+  }
+  __syncthreads();
+  unsigned written = 0, eq_seen = 0;  // selected tokens and ties of theta before this warp's segment
+  for (int w = 0; w < warp; ++w) {
+    const unsigned eq_take = eq_seen < take_eq ? min(s_eq[w], take_eq - eq_seen) : 0u;
+    written += s_gt[w] + eq_take;
+    eq_seen += s_eq[w];
+  }
+  const unsigned below = (1u << lane) - 1u;
+  for (int base = s0; base < s1; base += 32) {
+    const int t = base + lane;
+    const unsigned u = t < s1 ? __float_as_uint(__ldg(e + t)) : 0u;
+    const bool gt = t < s1 && u > theta;
+    const bool eq = t < s1 && u == theta;
+    const unsigned eq_bal = __ballot_sync(0xffffffffu, eq);
+    const bool sel = gt || (eq && eq_seen + __popc(eq_bal & below) < take_eq);
+    const unsigned sel_bal = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[written + __popc(sel_bal & below)] = t;
+    written += __popc(sel_bal);
+    eq_seen += __popc(eq_bal);
   }
 }
 
