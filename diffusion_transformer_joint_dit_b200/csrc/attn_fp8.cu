@@ -340,6 +340,9 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float c1 = sq * __ldg(prm.k_scale + scale_row + kb1);
       const float sv0 = __ldg(prm.v_scale + scale_row + kb0);
       const float sv1 = __ldg(prm.v_scale + scale_row + kb1);
+      // Per-half constants that do not depend on S, formed before the wait.
+      const float lb0 = __log2f(sv0) - lg_norm, lb1 = __log2f(sv1) - lg_norm;
+      const float vi0 = v_norm / sv0, vi1 = v_norm / sv1;
       if (!__all_sync(0xffffffffu,
                       mbar_wait(&ctrl->s_full[t], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns))) {
         ok = false;
@@ -374,12 +377,12 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         m = mnew;
       }
       // Exponent biases fold the V block scales: P' = P * sv / 2^e.
-      const float bias0 = __log2f(sv0) - lg_norm - m;
-      const float bias1 = __log2f(sv1) - lg_norm - m;
+      const float bias0 = lb0 - m;
+      const float bias1 = lb1 - m;
       float l0, l1;
       exp_pack_tile<true, kPolyEvery, false>(sv, c0, bias0, c1, bias1, nvalid >= kBN, l0, l1);
       // Undo the V-scale fold for the row sum: sum P = sum P' * 2^e / sv.
-      l += l0 * (v_norm / sv0) + (nvalid > 64 ? l1 * (v_norm / sv1) : 0.f);
+      l += l0 * vi0 + (nvalid > 64 ? l1 * vi1 : 0.f);
       tmem_st32(s_addr, sv[0]);
       tmem_st32(s_addr + 32, sv[2]);
       // O correction after P is out of registers (keeps register pressure

@@ -181,3 +181,46 @@ def test_t2i_2048_tau_1_sampled(cuda_ok):
     assert np.max(np.abs(got - ref)) <= BF16_MAX_ABS
     assert np.max(np.abs(to_np(lse)[:, :, rows] - ref_lse)) <= BF16_LSE_ABS
     print(f"t2i_2048 tau=1.0: kept {keep.mean():.3f} of the key blocks")
+
+
+def test_select_on_a_sequence_that_needs_more_shared_memory(cuda_ok):
+    """Key-block scores live in shared memory (4 B per key block): two
+    calls whose sequences need more than 48 KB, the second more than the
+    first, both launch (the kernel's shared-memory limit is raised again).
+    Checked on sampled query blocks against the oracle's rule applied to the
+    kernel's probabilities and against pooled means recomputed here."""
+    B, H, d = 1, 1, 128
+    for n in (1_600_000, 2_000_000):
+        g = torch.Generator(device="cuda").manual_seed(n)
+        q = torch.randn((B, n, H, d), generator=g, device="cuda").to(torch.bfloat16)
+        k = torch.randn((B, n, H, d), generator=g, device="cuda").to(torch.bfloat16)
+        nqb, nkb = J.sparse_blocks(n)
+        assert nkb * 4 > 48 * 1024
+        qbar = torch.empty((B, H, nqb, d), dtype=torch.float32, device="cuda")
+        kbar = torch.empty((B, H, nkb, d), dtype=torch.float32, device="cuda")
+        idx = torch.empty((B, H, nqb, nkb), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((B, H, nqb), dtype=torch.int32, device="cuda")
+        scale = 0.0883883
+        J.jattn_sparse_select(q, k, qbar, kbar, None, idx, cnt, B, H, n, 0, 0, d, scale, 1.0)
+        torch.cuda.synchronize()
+        # Pooled means of a few blocks, recomputed from the tensors (float64).
+        for i in (0, nkb // 2, nkb - 1):
+            ref = k[0, i * 128:(i + 1) * 128, 0].double().mean(0)
+            assert torch.allclose(kbar[0, 0, i].double(), ref, atol=2e-6 * float(k.abs().max()))
+        # The kept lists of sampled query blocks: the rule on probabilities
+        # formed here in float64 from the kernel's pooled means.
+        kb = kbar[0, 0].double()
+        for i in (0, nqb // 3, nqb - 1):
+            s = scale * (kb @ qbar[0, 0, i].double())
+            p = torch.softmax(s, 0).cpu().numpy()
+            c = int(cnt[0, 0, i])
+            row = to_np(idx[0, 0, i, :c]).astype(np.int64)
+            assert c >= 1 and np.all(np.diff(row) > 0)
+            # Blocks clearly above or below the threshold agree with the rule.
+            thr = 1.0 / nkb
+            clear_in = np.nonzero(p >= thr * (1 + 1e-3))[0]
+            clear_out = np.nonzero(p < thr * (1 - 1e-3))[0]
+            assert set(clear_in.tolist()) <= set(row.tolist())
+            assert not (set(clear_out.tolist()) & set(row.tolist()) - {int(np.argmax(p))})
+        del q, k, idx
+        torch.cuda.empty_cache()
