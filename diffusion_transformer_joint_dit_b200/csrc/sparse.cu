@@ -50,27 +50,17 @@ sparse_pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
     const size_t stride = static_cast<size_t>(H) * kD;
     const __nv_bfloat16* qp = q + (static_cast<size_t>(b) * N * H + h) * kD + c8;
     const __nv_bfloat16* kp = k + (static_cast<size_t>(b) * N * H + h) * kD + c8;
-    // Batches of 8 tokens: 16 loads in flight per thread before any is used.
-    constexpr int kBatch = 8;
-    for (int tb = t0; tb < t1; tb += kBatch) {
-      uint4 a[kBatch], c[kBatch];
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(qp + t * stride));
+      const uint4 c = __ldg(reinterpret_cast<const uint4*>(kp + t * stride));
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int t = min(tb + u, t1 - 1);
-        a[u] = __ldg(reinterpret_cast<const uint4*>(qp + t * stride));
-        c[u] = __ldg(reinterpret_cast<const uint4*>(kp + t * stride));
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        if (tb + u >= t1) break;  // in token order, as the sums are defined
-        const uint32_t aw[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, cw[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          sq[2 * i] += __uint_as_float(aw[i] << 16);
-          sq[2 * i + 1] += __uint_as_float(aw[i] & 0xFFFF0000u);
-          sk[2 * i] += __uint_as_float(cw[i] << 16);
-          sk[2 * i + 1] += __uint_as_float(cw[i] & 0xFFFF0000u);
-        }
+      for (int i = 0; i < 4; ++i) {
+        sq[2 * i] += __uint_as_float(aw[i] << 16);
+        sq[2 * i + 1] += __uint_as_float(aw[i] & 0xFFFF0000u);
+        sk[2 * i] += __uint_as_float(cw[i] << 16);
+        sk[2 * i + 1] += __uint_as_float(cw[i] & 0xFFFF0000u);
       }
     }
   }
