@@ -77,7 +77,7 @@ def rmsnorm(x, w=None, eps: float = 1e-6) -> np.ndarray:
 
 
 def token_positions(n_txt: int, img_h: int, img_w: int,
-                    ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0):
+                    ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0, ref_grids=None):
     """(row, col) RoPE positions of the joint sequence [text | image | ref].
 
     Text tokens sit at (0, 0).  Image token t' (0-based within the image
@@ -85,17 +85,30 @@ def token_positions(n_txt: int, img_h: int, img_w: int,
     flattened row-major.  Reference token t'' sits at
     (ref_row_offset + t'' // ref_w, t'' % ref_w): the reference grid is a
     second grid shifted down by ``ref_row_offset`` rows.
+
+    Several reference images (the tutorial's editing command repeats
+    ``--image`` for multiple references; the pages give no position rule
+    for them): ``ref_grids`` lists one ``(h, w, row_offset, col_offset)``
+    per reference, in sequence order, and replaces ref_h / ref_w /
+    ref_row_offset.  Token u of reference g sits at
+    (row_offset_g + u // w_g, col_offset_g + u % w_g).  One grid
+    ``(ref_h, ref_w, ref_row_offset, 0)`` is the single-reference rule.
     """
+    if ref_grids is None:
+        ref_grids = [(ref_h, ref_w, ref_row_offset, 0)] if ref_h * ref_w > 0 else []
     n_img = img_h * img_w
-    n_ref = ref_h * ref_w
+    n_ref = sum(h * w for h, w, _, _ in ref_grids)
     rows = np.zeros(n_txt + n_img + n_ref, dtype=np.int64)
     cols = np.zeros_like(rows)
     for t in range(n_img):
         rows[n_txt + t] = t // img_w
         cols[n_txt + t] = t % img_w
-    for t in range(n_ref):
-        rows[n_txt + n_img + t] = ref_row_offset + t // ref_w
-        cols[n_txt + n_img + t] = t % ref_w
+    start = n_txt + n_img
+    for h, w, row0, col0 in ref_grids:
+        for u in range(h * w):
+            rows[start + u] = row0 + u // w
+            cols[start + u] = col0 + u % w
+        start += h * w
     return rows, cols
 
 
@@ -131,7 +144,7 @@ def rope_2d(x, pos_row, pos_col, theta: float = 10000.0) -> np.ndarray:
 
 
 def prologue(q, k, *, n_txt: int, img_h: int, img_w: int,
-             ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0,
+             ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0, ref_grids=None,
              theta: float = 10000.0, eps: float = 1e-6,
              q_norm_w=None, k_norm_w=None):
     """Q' = RoPE(RMSNorm(Q)), K' = RoPE(RMSNorm(K)), in float64.
@@ -140,14 +153,14 @@ def prologue(q, k, *, n_txt: int, img_h: int, img_w: int,
     optimization" section lists them.  V passes through untouched.  Inputs
     ``[B, N, H, d]``; returns unrounded float64 arrays of the same shape.
     """
-    rows, cols = token_positions(n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset)
+    rows, cols = token_positions(n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset, ref_grids)
     qn = rmsnorm(q, q_norm_w, eps)
     kn = rmsnorm(k, k_norm_w, eps)
     return rope_2d(qn, rows, cols, theta), rope_2d(kn, rows, cols, theta)
 
 
 def rope_table(n_txt: int, img_h: int, img_w: int, ref_h: int = 0, ref_w: int = 0,
-               ref_row_offset: int = 0, theta: float = 10000.0) -> np.ndarray:
+               ref_row_offset: int = 0, ref_grids=None, theta: float = 10000.0) -> np.ndarray:
     """(cos, sin) of every token's 64 rotation angles, ``[N, 64, 2]`` float64.
 
     Entry (t, j): angle pos * theta**(-2 (j mod 32) / 64) with pos the row
@@ -155,7 +168,7 @@ def rope_table(n_txt: int, img_h: int, img_w: int, ref_h: int = 0, ref_w: int = 
     the angle ``rope_2d`` applies to channel pair (2j, 2j+1) of a 128-wide
     head.
     """
-    rows, cols = token_positions(n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset)
+    rows, cols = token_positions(n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset, ref_grids)
     n = len(rows)
     out = np.empty((n, 64, 2), dtype=np.float64)
     for j in range(64):
@@ -167,7 +180,7 @@ def rope_table(n_txt: int, img_h: int, img_w: int, ref_h: int = 0, ref_w: int = 
 
 
 def qkv_fused(x, w_txt, w_img, *, n_txt: int, img_h: int, img_w: int, H: int,
-              ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0,
+              ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0, ref_grids=None,
               theta: float = 10000.0, eps: float = 1e-6,
               q_norm_w=(None, None), k_norm_w=(None, None)):
     """QKV projection with the prologue in its epilogue, in float64.
@@ -197,7 +210,7 @@ def qkv_fused(x, w_txt, w_img, *, n_txt: int, img_h: int, img_w: int, H: int,
     for s, sl in ((0, slice(0, n_txt)), (1, slice(n_txt, N))):
         qn[:, sl] = rmsnorm(q[:, sl], q_norm_w[s], eps)
         kn[:, sl] = rmsnorm(k[:, sl], k_norm_w[s], eps)
-    rows, cols = token_positions(n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset)
+    rows, cols = token_positions(n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset, ref_grids)
     return rope_2d(qn, rows, cols, theta), rope_2d(kn, rows, cols, theta), v
 
 

@@ -74,6 +74,37 @@ def test_token_positions_small_grid():
     assert list(cols) == [0, 0, 0, 1, 2, 0, 1, 2, 0, 1, 0, 1]
 
 
+def test_token_positions_several_reference_grids():
+    # Text 1, image 1 x 2, then a 2 x 1 reference at (5, 3) and a 1 x 2 one at (7, 0).
+    rows, cols = O.token_positions(1, 1, 2, ref_grids=[(2, 1, 5, 3), (1, 2, 7, 0)])
+    assert list(rows) == [0, 0, 0, 5, 6, 7, 7]
+    assert list(cols) == [0, 0, 1, 3, 3, 0, 1]
+    # One grid at column 0 is the single-reference rule.
+    r1, c1 = O.token_positions(2, 2, 3, ref_h=2, ref_w=2, ref_row_offset=2)
+    r2, c2 = O.token_positions(2, 2, 3, ref_grids=[(2, 2, 2, 0)])
+    assert list(r1) == list(r2) and list(c1) == list(c2)
+
+
+def test_shifting_one_reference_grid_keeps_its_own_scores():
+    # RoPE scores depend on position differences only: moving a whole
+    # reference grid leaves the scores among its own tokens unchanged and
+    # changes those against the other streams.
+    rng = np.random.default_rng(12)
+    n_txt, img_h, img_w = 2, 2, 3
+    grids_a = [(2, 2, 2, 0), (1, 3, 4, 0)]
+    grids_b = [(2, 2, 2, 0), (1, 3, 9, 5)]
+    N = n_txt + img_h * img_w + 4 + 3
+    q = rng.standard_normal((1, N, 1, 128))
+    k = rng.standard_normal((1, N, 1, 128))
+    out = []
+    for g in (grids_a, grids_b):
+        qp, kp = O.prologue(q, k, n_txt=n_txt, img_h=img_h, img_w=img_w, ref_grids=g)
+        out.append(qp[0, :, 0] @ kp[0, :, 0].T)
+    own = slice(N - 3, N)
+    np.testing.assert_allclose(out[0][own, own], out[1][own, own], rtol=1e-12, atol=1e-12)
+    assert np.max(np.abs(out[0][own, :n_txt + 6] - out[1][own, :n_txt + 6])) > 1e-3
+
+
 # ----------------------------------------------------------------- RoPE ----
 
 def _unit(ch, d=128):
