@@ -26,6 +26,7 @@ JATTN_ERR_TIMEOUT = 5
 JATTN_PROLOGUE_BF16 = 0
 JATTN_PROLOGUE_FP8 = 1
 JATTN_FP8_BLOCK = 64
+JATTN_MAX_REF_GRIDS = 8
 JATTN_SPARSE_QBLOCK = 256
 JATTN_SPARSE_KBLOCK = 128
 
@@ -44,6 +45,10 @@ class JattnError(RuntimeError):
         super().__init__(msg)
 
 
+class jattn_ref_grid(ctypes.Structure):
+    _fields_ = [("h", ctypes.c_int), ("w", ctypes.c_int), ("row_offset", ctypes.c_int), ("col_offset", ctypes.c_int)]
+
+
 class jattn_prologue_params(ctypes.Structure):
     _fields_ = [
         ("img_h", ctypes.c_int), ("img_w", ctypes.c_int),
@@ -51,6 +56,7 @@ class jattn_prologue_params(ctypes.Structure):
         ("ref_row_offset", ctypes.c_int),
         ("rope_theta", ctypes.c_float), ("eps", ctypes.c_float),
         ("q_norm_w", ctypes.c_void_p), ("k_norm_w", ctypes.c_void_p),
+        ("n_ref_grids", ctypes.c_int), ("ref_grids", ctypes.POINTER(jattn_ref_grid)),
     ]
 
 
@@ -145,9 +151,19 @@ def jattn_status_string(status: int) -> str:
 
 
 def make_prologue_params(img_h: int, img_w: int, ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0,
-                         rope_theta: float = 10000.0, eps: float = 1e-6, q_norm_w=None, k_norm_w=None):
-    return jattn_prologue_params(img_h, img_w, ref_h, ref_w, ref_row_offset, rope_theta, eps,
-                                 _ptr(q_norm_w), _ptr(k_norm_w))
+                         rope_theta: float = 10000.0, eps: float = 1e-6, q_norm_w=None, k_norm_w=None,
+                         ref_grids=None):
+    """Prologue parameters.  ``ref_grids``: optional sequence of
+    ``(h, w, row_offset, col_offset)``, one per reference image, in sequence
+    order; it replaces ref_h / ref_w / ref_row_offset."""
+    p = jattn_prologue_params(img_h, img_w, ref_h, ref_w, ref_row_offset, rope_theta, eps,
+                              _ptr(q_norm_w), _ptr(k_norm_w), 0, None)
+    if ref_grids:
+        arr = (jattn_ref_grid * len(ref_grids))(*[jattn_ref_grid(*g) for g in ref_grids])
+        p.n_ref_grids = len(ref_grids)
+        p.ref_grids = ctypes.cast(arr, ctypes.POINTER(jattn_ref_grid))
+        p._grids_keepalive = arr  # the host array must outlive the calls that read it
+    return p
 
 
 def jattn_prologue(q, k, v, q_out, k_out, v_out, q_scale, k_scale, v_scale,

@@ -90,6 +90,51 @@ int check_common(int B, int H, int N_txt, int N_img, int N_ref, int d) {
   return JATTN_OK;
 }
 
+// Validates the position and RoPE parameters against the stream sizes and
+// fills the position fields and frequencies of `a`; returns a jattn_status.
+static_assert(JATTN_MAX_REF_GRIDS == kMaxRefGrids, "reference-grid limit");
+
+int fill_positions(PrologueArgs& a, const jattn_prologue_params* p, int N_txt, int N_img, int N_ref) {
+  if (p == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (p->img_h < 0 || p->img_w < 0 || static_cast<long long>(p->img_h) * p->img_w != N_img)
+    return JATTN_ERR_INVALID_ARG;
+  if (!(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta)) return JATTN_ERR_INVALID_ARG;
+  a.n_txt = N_txt;
+  a.n_img = N_img;
+  a.img_w = p->img_w > 0 ? p->img_w : 1;
+  a.n_grids = 0;
+  if (p->n_ref_grids == 0) {
+    if (p->ref_h < 0 || p->ref_w < 0 || p->ref_row_offset < 0 ||
+        static_cast<long long>(p->ref_h) * p->ref_w != N_ref)
+      return JATTN_ERR_INVALID_ARG;
+    if (N_ref > 0) {
+      a.n_grids = 1;
+      a.grid_end[0] = N_ref;
+      a.grid_w[0] = p->ref_w;
+      a.grid_row[0] = p->ref_row_offset;
+      a.grid_col[0] = 0;
+    }
+  } else {
+    if (p->n_ref_grids < 0 || p->n_ref_grids > JATTN_MAX_REF_GRIDS || p->ref_grids == nullptr)
+      return JATTN_ERR_INVALID_ARG;
+    long long end = 0;
+    for (int g = 0; g < p->n_ref_grids; ++g) {
+      const jattn_ref_grid& r = p->ref_grids[g];
+      if (r.h < 1 || r.w < 1 || r.row_offset < 0 || r.col_offset < 0) return JATTN_ERR_INVALID_ARG;
+      end += static_cast<long long>(r.h) * r.w;
+      if (end > N_ref) return JATTN_ERR_INVALID_ARG;
+      a.grid_end[g] = static_cast<int>(end);
+      a.grid_w[g] = r.w;
+      a.grid_row[g] = r.row_offset;
+      a.grid_col[g] = r.col_offset;
+    }
+    if (end != N_ref) return JATTN_ERR_INVALID_ARG;
+    a.n_grids = p->n_ref_grids;
+  }
+  for (int i = 0; i < 32; ++i) a.omega[i] = std::pow(static_cast<double>(p->rope_theta), -2.0 * i / 64.0);
+  return JATTN_OK;
+}
+
 }  // namespace
 
 cudaError_t make_act_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int elem_bytes) {
@@ -212,12 +257,10 @@ int jattn_prologue(const void* q, const void* k, const void* v, void* q_out, voi
   int st = check_common(B, H, N_txt, N_img, N_ref, d);
   if (st != JATTN_OK) return st;
   if (p == nullptr || (mode != JATTN_PROLOGUE_BF16 && mode != JATTN_PROLOGUE_FP8)) return JATTN_ERR_INVALID_ARG;
-  if (p->img_h < 0 || p->img_w < 0 || p->ref_h < 0 || p->ref_w < 0 || p->ref_row_offset < 0)
-    return JATTN_ERR_INVALID_ARG;
-  if (static_cast<long long>(p->img_h) * p->img_w != N_img || static_cast<long long>(p->ref_h) * p->ref_w != N_ref)
-    return JATTN_ERR_INVALID_ARG;
-  if (!(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta) || !(p->eps >= 0.f) || !std::isfinite(p->eps))
-    return JATTN_ERR_INVALID_ARG;
+  PrologueArgs a;
+  std::memset(&a, 0, sizeof(a));
+  if ((st = fill_positions(a, p, N_txt, N_img, N_ref)) != JATTN_OK) return st;
+  if (!(p->eps >= 0.f) || !std::isfinite(p->eps)) return JATTN_ERR_INVALID_ARG;
   if (q == nullptr || k == nullptr || q_out == nullptr || k_out == nullptr) return JATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return JATTN_ERR_MISALIGNED;
   if (!aligned16(p->q_norm_w) || !aligned16(p->k_norm_w)) return JATTN_ERR_MISALIGNED;
@@ -229,20 +272,13 @@ int jattn_prologue(const void* q, const void* k, const void* v, void* q_out, voi
          reinterpret_cast<uintptr_t>(v_scale)) & 3u)
       return JATTN_ERR_MISALIGNED;
   }
-  PrologueArgs a;
-  std::memset(&a, 0, sizeof(a));
   a.q = q; a.k = k; a.v = v;
   a.q_out = q_out; a.k_out = k_out; a.v_out = v_out;
   a.q_scale = q_scale; a.k_scale = k_scale; a.v_scale = v_scale;
   a.q_w = p->q_norm_w; a.k_w = p->k_norm_w;
   a.B = B; a.H = H; a.N = N_txt + N_img + N_ref;
-  a.n_txt = N_txt; a.n_img = N_img;
-  a.img_w = p->img_w > 0 ? p->img_w : 1;
-  a.ref_w = p->ref_w > 0 ? p->ref_w : 1;
-  a.ref_row_offset = p->ref_row_offset;
   a.eps = p->eps;
   a.timeout_ns = kDefaultTimeoutNs;
-  for (int i = 0; i < 32; ++i) a.omega[i] = std::pow(static_cast<double>(p->rope_theta), -2.0 * i / 64.0);
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   return map_err(mode == JATTN_PROLOGUE_BF16 ? launch_prologue_bf16(a, s) : launch_prologue_fp8(a, s));
 }
@@ -342,19 +378,10 @@ int jattn_rope_table(float* table, int N_txt, int N_img, int N_ref, const jattn_
   if (st != JATTN_OK) return st;
   if (table == nullptr || p == nullptr) return JATTN_ERR_INVALID_ARG;
   if (!aligned16(table)) return JATTN_ERR_MISALIGNED;
-  if (p->img_h < 0 || p->img_w < 0 || p->ref_h < 0 || p->ref_w < 0 || p->ref_row_offset < 0)
-    return JATTN_ERR_INVALID_ARG;
-  if (static_cast<long long>(p->img_h) * p->img_w != N_img || static_cast<long long>(p->ref_h) * p->ref_w != N_ref)
-    return JATTN_ERR_INVALID_ARG;
-  if (!(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta)) return JATTN_ERR_INVALID_ARG;
   PrologueArgs a;
   std::memset(&a, 0, sizeof(a));
+  if ((st = fill_positions(a, p, N_txt, N_img, N_ref)) != JATTN_OK) return st;
   a.B = 1; a.H = 1; a.N = N_txt + N_img + N_ref;
-  a.n_txt = N_txt; a.n_img = N_img;
-  a.img_w = p->img_w > 0 ? p->img_w : 1;
-  a.ref_w = p->ref_w > 0 ? p->ref_w : 1;
-  a.ref_row_offset = p->ref_row_offset;
-  for (int i = 0; i < 32; ++i) a.omega[i] = std::pow(static_cast<double>(p->rope_theta), -2.0 * i / 64.0);
   return map_err(launch_rope_table(a, table, static_cast<cudaStream_t>(cuda_stream)));
 }
 
@@ -397,25 +424,16 @@ namespace {
 // by jattn_prologue and the repair selection; returns a jattn_status.
 int fill_prologue_args(PrologueArgs& a, const void* q, const void* k, const void* v, int B, int H, int N_txt,
                        int N_img, int N_ref, const jattn_prologue_params* p) {
-  if (p == nullptr) return JATTN_ERR_INVALID_ARG;
-  if (p->img_h < 0 || p->img_w < 0 || p->ref_h < 0 || p->ref_w < 0 || p->ref_row_offset < 0)
-    return JATTN_ERR_INVALID_ARG;
-  if (static_cast<long long>(p->img_h) * p->img_w != N_img || static_cast<long long>(p->ref_h) * p->ref_w != N_ref)
-    return JATTN_ERR_INVALID_ARG;
-  if (!(p->rope_theta > 0.f) || !std::isfinite(p->rope_theta) || !(p->eps >= 0.f) || !std::isfinite(p->eps))
-    return JATTN_ERR_INVALID_ARG;
-  if (!aligned16(p->q_norm_w) || !aligned16(p->k_norm_w)) return JATTN_ERR_MISALIGNED;
   std::memset(&a, 0, sizeof(a));
+  const int st = fill_positions(a, p, N_txt, N_img, N_ref);
+  if (st != JATTN_OK) return st;
+  if (!(p->eps >= 0.f) || !std::isfinite(p->eps)) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(p->q_norm_w) || !aligned16(p->k_norm_w)) return JATTN_ERR_MISALIGNED;
   a.q = q; a.k = k; a.v = v;
   a.q_w = p->q_norm_w; a.k_w = p->k_norm_w;
   a.B = B; a.H = H; a.N = N_txt + N_img + N_ref;
-  a.n_txt = N_txt; a.n_img = N_img;
-  a.img_w = p->img_w > 0 ? p->img_w : 1;
-  a.ref_w = p->ref_w > 0 ? p->ref_w : 1;
-  a.ref_row_offset = p->ref_row_offset;
   a.eps = p->eps;
   a.timeout_ns = kDefaultTimeoutNs;
-  for (int i = 0; i < 32; ++i) a.omega[i] = std::pow(static_cast<double>(p->rope_theta), -2.0 * i / 64.0);
   return JATTN_OK;
 }
 

@@ -11,6 +11,7 @@ namespace jattn {
 
 constexpr int kHeadDim = 128;
 constexpr int kQuantBlock = 64;
+constexpr int kMaxRefGrids = 8;
 
 // Arguments of the prologue kernels, passed by value (__grid_constant__).
 struct PrologueArgs {
@@ -26,7 +27,15 @@ struct PrologueArgs {
   const float* q_w;  // nullable: weight 1.0
   const float* k_w;
   int B, H, N;
-  int n_txt, n_img, img_w, ref_w, ref_row_offset;
+  int n_txt, n_img, img_w;
+  // Reference grids in sequence order: grid g covers reference tokens
+  // [grid_end[g - 1], grid_end[g]) (grid_end[-1] = 0), row-major with width
+  // grid_w[g], placed at (grid_row[g], grid_col[g]).
+  int n_grids;
+  int grid_end[kMaxRefGrids];
+  int grid_w[kMaxRefGrids];
+  int grid_row[kMaxRefGrids];
+  int grid_col[kMaxRefGrids];
   float eps;
   uint64_t timeout_ns;  // bound of each barrier wait (FP8 mode)
   // RoPE frequencies of the 32 channel pairs of one axis half,

@@ -17,29 +17,13 @@
 #include <cuda_fp8.h>
 
 #include "jattn_internal.h"
+#include "positions.cuh"
 #include "sm100_ptx.cuh"
 #include "softmax_sm100.cuh"
 
 namespace jattn {
 
 namespace {
-
-// (row, col) RoPE position of joint-sequence token t.
-__device__ __forceinline__ void token_pos(const PrologueArgs& a, int t, int& row, int& col) {
-  if (t < a.n_txt) {
-    row = 0;
-    col = 0;
-  } else if (t < a.n_txt + a.n_img) {
-    const int u = t - a.n_txt;
-    row = u / a.img_w;
-    col = u - row * a.img_w;
-  } else {
-    const int u = t - a.n_txt - a.n_img;
-    const int r = u / a.ref_w;
-    row = a.ref_row_offset + r;
-    col = u - r * a.ref_w;
-  }
-}
 
 // cos / sin of pos * omega for the lane's 4 channel pairs.  The angle is
 // formed and reduced to [-pi, pi] in double, then evaluated in float.

@@ -27,6 +27,7 @@
 // loop (first pass over TMEM), the scaling, weights and rotation a second
 // pass, 32 channels at a time.
 #include "jattn_internal.h"
+#include "positions.cuh"
 #include "sm100_ptx.cuh"
 
 namespace jattn {
@@ -384,19 +385,8 @@ __global__ void rope_table_kernel(const __grid_constant__ PrologueArgs a, float2
   const long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (e >= static_cast<long long>(a.N) * 64) return;
   const int t = static_cast<int>(e >> 6), pr = static_cast<int>(e & 63);
-  int row = 0, col = 0;
-  if (t < a.n_txt) {
-    row = col = 0;
-  } else if (t < a.n_txt + a.n_img) {
-    const int u = t - a.n_txt;
-    row = u / a.img_w;
-    col = u - row * a.img_w;
-  } else {
-    const int u = t - a.n_txt - a.n_img;
-    const int rr = u / a.ref_w;
-    row = a.ref_row_offset + rr;
-    col = u - rr * a.ref_w;
-  }
+  int row, col;
+  token_pos(a, t, row, col);
   constexpr double kTwoPi = 6.283185307179586476925286766559;
   constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
   const double phi = static_cast<double>(pr < 32 ? row : col) * a.omega[pr & 31];

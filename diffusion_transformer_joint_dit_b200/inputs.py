@@ -32,6 +32,7 @@ class Workload:
     ref_h: int = 0
     ref_w: int = 0
     ref_row_offset: int = 0
+    ref_grids: tuple = ()         # several references: ((h, w, row_offset, col_offset), ...)
     d: int = 128
     path: str = "bf16"            # "bf16" or "fp8"
     k_outlier_frac: float = 0.0   # fraction of K' rows scaled by k_outlier_gain
@@ -48,6 +49,8 @@ class Workload:
 
     @property
     def n_ref(self) -> int:
+        if self.ref_grids:
+            return sum(h * w for h, w, _, _ in self.ref_grids)
         return self.ref_h * self.ref_w
 
     @property

@@ -81,9 +81,25 @@ typedef enum {
  * position; inside a half, adjacent pair (2i, 2i+1) rotates by
  * pos * rope_theta^(-2i/(d/2)).
  *
+ * Several reference images (the tutorial's editing command takes one
+ * --image per reference; the pages give no position rule for them): with
+ * n_ref_grids > 0, the reference stream is the concatenation of
+ * n_ref_grids grids in the order of ref_grids, token u of grid g at
+ * (row_offset_g + u / w_g, col_offset_g + u % w_g), and ref_h, ref_w,
+ * ref_row_offset are ignored; N_ref must equal the sum of h_g * w_g.  One
+ * grid {ref_h, ref_w, ref_row_offset, 0} is the single-reference rule.
+ *
  * RMSNorm: y = x / sqrt(mean_c(x^2) + eps) * w[c], per (b, t, h), fp32 math.
  * q_norm_w / k_norm_w are device pointers to d fp32 weights, or NULL for 1.0.
  */
+#define JATTN_MAX_REF_GRIDS 8
+
+typedef struct {
+  int h, w;                /* grid size, each >= 1 */
+  int row_offset;          /* position of the grid's first row, >= 0 */
+  int col_offset;          /* position of the grid's first column, >= 0 */
+} jattn_ref_grid;
+
 typedef struct {
   int img_h, img_w;        /* noisy-target latent grid; N_img must equal img_h * img_w */
   int ref_h, ref_w;        /* reference grid; N_ref must equal ref_h * ref_w (0 x 0 = none) */
@@ -92,6 +108,8 @@ typedef struct {
   float eps;               /* RMSNorm epsilon, >= 0 (workloads: 1e-6) */
   const float* q_norm_w;   /* [d] fp32 device pointer or NULL */
   const float* k_norm_w;   /* [d] fp32 device pointer or NULL */
+  int n_ref_grids;         /* 0: the single grid above; 1 .. JATTN_MAX_REF_GRIDS: ref_grids */
+  const jattn_ref_grid* ref_grids;  /* host array of n_ref_grids grids, or NULL */
 } jattn_prologue_params;
 
 /*

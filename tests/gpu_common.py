@@ -30,7 +30,8 @@ def to_np(t: torch.Tensor) -> np.ndarray:
 
 
 def prologue_params(w: I.Workload):
-    return J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps)
+    return J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps,
+                                  ref_grids=w.ref_grids or None)
 
 
 def gpu_prologue_bf16(w: I.Workload, q, k):
@@ -68,7 +69,7 @@ def oracle_prologue_bf16(w: I.Workload, q, k):
     """Oracle Q', K' (float64) and their bf16 roundings (float64 arrays)."""
     qp, kp = O.prologue(to_np(q), to_np(k), n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w,
                         ref_h=w.ref_h, ref_w=w.ref_w, ref_row_offset=w.ref_row_offset,
-                        theta=w.theta, eps=w.eps)
+                        ref_grids=list(w.ref_grids) or None, theta=w.theta, eps=w.eps)
     return qp, kp, O.bf16_round(qp), O.bf16_round(kp)
 
 

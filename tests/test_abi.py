@@ -106,6 +106,22 @@ def test_prologue_rejects_bad_arguments(lib, kw, status):
     assert prologue(**kw) == status
 
 
+def test_reference_grids_are_validated(lib):
+    # 32 text + 16 x 16 image + references of 2 x 16 and 1 x 8 = 40 tokens.
+    call = lambda grids, n_ref=40: prologue(N_ref=n_ref, params=J.make_prologue_params(16, 16, ref_grids=grids))
+    assert call([(2, 16, 16, 0), (1, 8, 18, 0)], n_ref=41) == J.JATTN_ERR_INVALID_ARG    # sizes do not add up
+    assert call([(2, 16, 16, 0), (0, 8, 18, 0)]) == J.JATTN_ERR_INVALID_ARG              # empty grid
+    assert call([(2, 16, -1, 0), (1, 8, 18, 0)]) == J.JATTN_ERR_INVALID_ARG              # negative offset
+    assert call([(2, 16, 16, 0), (1, 8, 18, -3)]) == J.JATTN_ERR_INVALID_ARG
+    assert call([(1, 4, 0, 0)] * 10) == J.JATTN_ERR_INVALID_ARG                           # more than 8 grids
+    p = J.make_prologue_params(16, 16)
+    p.n_ref_grids = 2                                                                      # no array
+    assert prologue(N_ref=40, params=p) == J.JATTN_ERR_INVALID_ARG
+    rope = lambda grids, n_ref: J.jattn_rope_table(A, 32, 256, n_ref, J.make_prologue_params(16, 16, ref_grids=grids),
+                                                   stream=0, check=False)
+    assert rope([(2, 16, 16, 0)], 31) == J.JATTN_ERR_INVALID_ARG
+
+
 def test_fwd_fp8_rejects_bad_arguments(lib):
     call = lambda **kw: J.jattn_fwd_fp8(
         kw.get("q", A), A, A, kw.get("qs", A), A, A, A, None, 1, 2, 32, 256, 0, kw.get("d", 128), 0.088,

@@ -29,6 +29,9 @@ EDGE = {
     "text_only_1": I.custom("text_only_1", B=1, H=1, n_txt=1, img_h=0, img_w=0),
     "rect_grid": I.custom("rect_grid", B=1, H=5, n_txt=3, img_h=7, img_w=13, ref_h=2, ref_w=9, ref_row_offset=7),
     "tail_block": I.custom("tail_block", B=1, H=2, n_txt=70, img_h=0, img_w=0),
+    # Three reference images, each with its own grid and (row, col) offsets.
+    "multi_ref": I.custom("multi_ref", B=2, H=3, n_txt=9, img_h=6, img_w=10,
+                          ref_grids=((4, 10, 6, 0), (3, 7, 10, 2), (2, 5, 0, 12))),
 }
 
 
@@ -45,7 +48,8 @@ def _bf16_close(got, exact):
     assert (d == 0).mean() >= 0.999, f"identical fraction {(d == 0).mean():.5f}"
 
 
-@pytest.mark.parametrize("name", ["tiny", "t2i_1024", "i2i_small", "text_only_1", "rect_grid", "tail_block"])
+@pytest.mark.parametrize("name", ["tiny", "t2i_1024", "i2i_small", "text_only_1", "rect_grid", "tail_block",
+                                  "multi_ref"])
 def test_prologue_bf16_matches_oracle(cuda_ok, name):
     w = I.WORKLOADS.get(name) or EDGE[name]
     q, k, _ = I.make_qkv(w, seed=3)
@@ -92,7 +96,7 @@ def _scales_close(got, ref):
     assert (got == ref).mean() >= 0.99
 
 
-@pytest.mark.parametrize("name", ["tiny", "i2i_small", "tail_block", "rect_grid", "t2i_2048_fp8"])
+@pytest.mark.parametrize("name", ["tiny", "i2i_small", "tail_block", "rect_grid", "multi_ref", "t2i_2048_fp8"])
 def test_prologue_fp8_matches_oracle(cuda_ok, name):
     w = I.WORKLOADS.get(name) or EDGE[name]
     q, k, v = I.make_qkv(w, seed=6)

@@ -30,6 +30,9 @@ CASES = {
     # No text tokens (text weights unused), K loop of 12 steps.
     "image_only": (I.custom("image_only", B=1, H=2, n_txt=0, img_h=9, img_w=15), 768),
     "text_only": (I.custom("text_only", B=1, H=2, n_txt=77, img_h=0, img_w=0), 192),
+    # Three reference grids with their own row and column offsets.
+    "multi_ref": (I.custom("multi_ref", B=1, H=2, n_txt=9, img_h=6, img_w=10,
+                           ref_grids=((4, 10, 6, 0), (3, 7, 10, 2), (2, 5, 0, 12))), 128),
 }
 
 
@@ -40,7 +43,8 @@ def _run(w, C, seed=0):
     qnd = [t.to(dev) for t in qn]
     knd = [t.to(dev) for t in kn]
     rope = torch.empty((w.N, 64, 2), dtype=torch.float32, device=dev)
-    params = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps)
+    params = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps,
+                                    ref_grids=w.ref_grids or None)
     J.jattn_rope_table(rope, w.n_txt, w.n_img, w.n_ref, params)
     shape = (w.B, w.N, w.H, w.d)
     q, k, v = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
@@ -71,11 +75,13 @@ def _check(got, exact, rotated):
 def test_qkv_fused_matches_oracle(cuda_ok, name):
     w, C = CASES[name]
     (x, wt, wi, qn, kn), rope, (q, k, v) = _run(w, C)
+    grids = list(w.ref_grids) or None
     np.testing.assert_allclose(rope, O.rope_table(w.n_txt, w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset,
-                                                  w.theta), rtol=0, atol=2e-7)
+                                                  grids, w.theta), rtol=0, atol=2e-7)
     f = lambda t: t.to(torch.float64).numpy()
     qe, ke, ve = O.qkv_fused(f(x), f(wt), f(wi), n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w, H=w.H,
-                             ref_h=w.ref_h, ref_w=w.ref_w, ref_row_offset=w.ref_row_offset, theta=w.theta,
+                             ref_h=w.ref_h, ref_w=w.ref_w, ref_row_offset=w.ref_row_offset, ref_grids=grids,
+                             theta=w.theta,
                              eps=w.eps, q_norm_w=tuple(t.numpy() for t in qn),
                              k_norm_w=tuple(t.numpy() for t in kn))
     _check(q, qe, True)

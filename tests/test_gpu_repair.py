@@ -50,11 +50,14 @@ CASES = {
     "ragged": I.custom("ragged", B=1, H=2, n_txt=7, img_h=9, img_w=21, gain_sigma=0.5),
     "two_batch": I.custom("two_batch", B=2, H=3, n_txt=5, img_h=8, img_w=8, ref_h=2, ref_w=8, ref_row_offset=8,
                           gain_sigma=0.5),
+    # Two reference grids: the exact K' rows are recomputed at their positions.
+    "multi_ref": I.custom("multi_ref", B=1, H=2, n_txt=6, img_h=8, img_w=9,
+                          ref_grids=((3, 9, 8, 0), (4, 5, 11, 9)), gain_sigma=0.5),
 }
 
 
 @pytest.mark.parametrize("name,m", [("ragged", 0), ("ragged", 1), ("ragged", 37), ("ragged", 196),
-                                    ("two_batch", 9)])
+                                    ("two_batch", 9), ("multi_ref", 11)])
 def test_repair_matches_oracle(cuda_ok, name, m):
     w = CASES[name]
     (q, k, v), codes, scales, (o0, lse0), (o, lse), err, idx, ksel, vsel = _run(w, m)
