@@ -145,12 +145,13 @@ def ulysses_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_total
 
 
 def jattn_bf16_ops(n_txt: int, n_img: int, n_ref: int, softmax_scale: float, img_h: int, img_w: int,
-                   ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0):
+                   ref_h: int = 0, ref_w: int = 0, ref_row_offset: int = 0, ref_grids=None):
     """(prologue, attn) for :func:`ulysses_attention` on CUDA tensors, both
-    through the jattn library (BF16 path)."""
+    through the jattn library (BF16 path).  ``ref_grids`` as for
+    ``binding.make_prologue_params`` (several reference images)."""
     from . import binding as J
 
-    params = J.make_prologue_params(img_h, img_w, ref_h, ref_w, ref_row_offset)
+    params = J.make_prologue_params(img_h, img_w, ref_h, ref_w, ref_row_offset, ref_grids=ref_grids)
 
     def prologue(q, k, v):
         b, n, h, d = q.shape
