@@ -21,12 +21,23 @@ __device__ __forceinline__ void token_pos(const PrologueArgs& a, int t, int& row
     return;
   }
   u -= a.n_img;
-  int g = 0;
-  while (g + 1 < a.n_grids && u >= a.grid_end[g]) ++g;
-  const int v = u - (g > 0 ? a.grid_end[g - 1] : 0);
-  const int r = v / a.grid_w[g];
-  row = a.grid_row[g] + r;
-  col = a.grid_col[g] + (v - r * a.grid_w[g]);
+  // The grid holding u, by a fixed-trip scan with constant indices (a
+  // data-dependent loop over the parameter arrays measured 8% slower in the
+  // FP8 prologue).
+  int start = 0, w = a.grid_w[0], row0 = a.grid_row[0], col0 = a.grid_col[0];
+#pragma unroll
+  for (int g = 1; g < kMaxRefGrids; ++g) {
+    if (g < a.n_grids && u >= a.grid_end[g - 1]) {
+      start = a.grid_end[g - 1];
+      w = a.grid_w[g];
+      row0 = a.grid_row[g];
+      col0 = a.grid_col[g];
+    }
+  }
+  const int v = u - start;
+  const int r = v / w;
+  row = row0 + r;
+  col = col0 + (v - r * w);
 }
 
 }  // namespace jattn
