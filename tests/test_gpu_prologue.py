@@ -106,3 +106,18 @@ def test_prologue_fp8_matches_oracle(cuda_ok, name):
         codes, scales = O.block_quantize_e4m3(x.astype(np.float32))
         _codes_close(got_c, codes)
         _scales_close(got_s, scales)
+
+
+@pytest.mark.parametrize("name", ["t2i_2048", "i2i_2048"])
+def test_prologue_bf16_full_size_sampled_tokens(cuda_ok, name):
+    """Full size, in the bench's launch configuration, checked on sampled
+    tokens (every head): the oracle's RMSNorm and 2-D RoPE applied to those
+    tokens at their positions in the whole sequence."""
+    w = I.WORKLOADS[name]
+    q, k, _ = I.make_qkv(w, seed=11)
+    qo, ko = gpu_prologue_bf16(w, q, k)
+    idx = I.sampled_rows(w, 256, seed=4)
+    rows, cols = O.token_positions(w.n_txt, w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset)
+    for got, x in ((qo, q), (ko, k)):
+        exact = O.rope_2d(O.rmsnorm(to_np(x[:, idx]), eps=w.eps), rows[idx], cols[idx], theta=w.theta)
+        _bf16_close(got[:, idx].cpu(), exact)
