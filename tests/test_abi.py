@@ -223,3 +223,13 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(J, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="not built"):
         J.load_library()
+
+
+def test_attention_api_rejects_bad_inputs_without_a_launch():
+    import torch
+    from diffusion_transformer_joint_dit_b200 import attention as A
+    x = torch.zeros((1, 4, 1, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        A.joint_attention(x, x, x, n_txt=4, img_h=0, img_w=0, config=A.AttentionConfig(mode="fp4"))
+    with pytest.raises(ValueError):
+        A.joint_attention(x, x, x, n_txt=4, img_h=0, img_w=0)      # CPU tensors
