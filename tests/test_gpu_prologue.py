@@ -96,7 +96,8 @@ def _scales_close(got, ref):
     assert (got == ref).mean() >= 0.99
 
 
-@pytest.mark.parametrize("name", ["tiny", "i2i_small", "tail_block", "rect_grid", "multi_ref", "t2i_2048_fp8"])
+@pytest.mark.parametrize("name", ["tiny", "i2i_small", "text_only_1", "tail_block", "rect_grid", "multi_ref",
+                                  "t2i_2048_fp8"])
 def test_prologue_fp8_matches_oracle(cuda_ok, name):
     w = I.WORKLOADS.get(name) or EDGE[name]
     q, k, v = I.make_qkv(w, seed=6)
