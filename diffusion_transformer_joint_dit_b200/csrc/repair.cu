@@ -2,8 +2,8 @@
 // quantisation lost the most are attended with their exact K' and V rows.
 //
 // The NVIDIA tutorial on FLUX 3 Image Klein ("Quantized and sparse
-// attention" section) runs VC-Attention FP8 with a repair budget rho that
-// selects the fraction of tokens with the highest quantisation error for
+// attention" section) runs VC-Attention FP8 with a repair budget rho: a
+// share rho of the tokens, those that quantisation hurt most, gets a
 // residual correction.  Reading implemented here, per (batch, head):
 //   error   e_t = |K'_t - Kd_t|^2 + |V_t - Vd_t|^2 (exact bf16 rows against
 //           their dequantised E4M3 values, fp32)            repair_error_kernel

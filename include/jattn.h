@@ -240,8 +240,8 @@ JATTN_API int jattn_qkv_fused(const void* x, const jattn_qkv_weights* w, const f
 
 /*
  * FP8 attention with a repair budget (the tutorial's VC-Attention FP8 runs
- * with a budget rho = 0.005 that "selects the fraction of tokens with the
- * highest quantisation error for residual correction"; "Quantized and
+ * with a budget rho = 0.005: a share rho of the tokens, those that
+ * quantisation hurt most, gets a residual correction; "Quantized and
  * sparse attention" section).  Reading implemented, per (batch, head):
  * the m tokens whose key and value rows lost the most in E4M3,
  *   e_t = sum_c (K'_tc - Kd_tc)^2 + sum_c (V_tc - Vd_tc)^2

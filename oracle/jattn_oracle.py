@@ -362,9 +362,9 @@ def repair_select(k_exact, v_exact, k_deq, v_deq, rho: float):
     """Key/value tokens with the highest quantisation error, per (b, h).
 
     The tutorial's "Quantized and sparse attention" section runs
-    VC-Attention FP8 with a repair budget rho = 0.005 that selects the
-    fraction of tokens with the highest quantisation error for residual
-    correction, without defining the error.  Reading: the error of token t
+    VC-Attention FP8 with a repair budget rho = 0.005: a share rho of the
+    tokens, those that quantisation hurt most, gets a residual correction.
+    The pages do not define the error.  Reading: the error of token t
     of (b, h) is the squared distance between its exact key and value rows
     (the bf16 K' and V the prologue quantises) and their dequantised E4M3
     values, summed over the d channels of both:
