@@ -208,9 +208,11 @@ def cpu_baseline(w: I.Workload, q, k, v, seconds: float):
         flops += oracle_unit(w, q, k, v, b, h, rows)
         done += 1
     dt = time.perf_counter() - t0
-    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    rate = flops / dt / 1e12
+    return {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": (f"float64 oracle (prologue of one (b,h) slice + attention of {rows_per_unit} sampled "
                        f"query rows vs all {w.N} keys) on {done} of {len(units)} (b,h) pairs, {dt:.1f} s"),
+            "full_step_s_extrapolated": w.flops / (rate * 1e12),
             "seconds": dt}
 
 
