@@ -33,7 +33,7 @@ JATTN_SPARSE_KBLOCK = 128
 EXPORTED = ("jattn_prologue", "jattn_fwd_bf16", "jattn_fwd_fp8", "jattn_rope_table", "jattn_qkv_fused",
             "jattn_fp8_repair_select", "jattn_fp8_repair_apply", "jattn_sparse_select", "jattn_fwd_bf16_sparse",
             "jattn_status_string", "jattn_device_status", "jattn_selftest_wait_timeout",
-            "jattn_selftest_exp2_poly", "jattn_last_cuda_error")
+            "jattn_selftest_exp2_poly", "jattn_last_cuda_error", "jattn_sparse_select_noalloc")
 
 
 class JattnError(RuntimeError):
@@ -106,6 +106,9 @@ def load_library():
     lib.jattn_sparse_select.restype = _I
     lib.jattn_fwd_bf16_sparse.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]
     lib.jattn_fwd_bf16_sparse.restype = _I
+    lib.jattn_sparse_select_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                                ctypes.c_float, ctypes.c_float, _P]
+    lib.jattn_sparse_select_noalloc.restype = _I
     lib.jattn_status_string.argtypes = [_I]
     lib.jattn_status_string.restype = ctypes.c_char_p
     lib.jattn_device_status.argtypes = [_P]
@@ -269,6 +272,18 @@ def jattn_sparse_select(q, k, qbar, kbar, probs, kv_idx, kv_cnt, B: int, H: int,
         B, H, N_txt, N_img, N_ref, d, softmax_scale, tau, _stream(stream))
     if check:
         _check("jattn_sparse_select", st)
+    return st
+
+
+def jattn_sparse_select_noalloc(q, k, probs, kv_idx, kv_cnt, B: int, H: int, N_txt: int, N_img: int, N_ref: int,
+                                d: int, softmax_scale: float, tau: float, stream=None, *, check: bool = True) -> int:
+    """jattn_sparse_select with the pooled-means workspace inside the library
+    (a fixed 16 MiB device array), for callers that cannot allocate."""
+    st = load_library().jattn_sparse_select_noalloc(
+        _ptr(q), _ptr(k), _ptr(probs), _ptr(kv_idx), _ptr(kv_cnt),
+        B, H, N_txt, N_img, N_ref, d, softmax_scale, tau, _stream(stream))
+    if check:
+        _check("jattn_sparse_select_noalloc", st)
     return st
 
 

@@ -519,3 +519,6 @@ int jattn_selftest_exp2_poly(const float* x, float* y, int n, void* cuda_stream)
 }
 
 }  // extern "C"
+
+// Entry point that needs no device allocation by the caller.
+#include "noalloc.cu"

@@ -354,6 +354,40 @@ JATTN_API int jattn_fwd_bf16_sparse(const void* q, const void* k, const void* v,
                           int B, int H, int N_txt, int N_img, int N_ref, int d,
                           float softmax_scale, void* cuda_stream);
 
+/*
+ * jattn_sparse_select_noalloc — jattn_sparse_select for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a service
+ * of the library, not a step of the method.
+ *
+ * Some callers cannot call cudaMalloc where they select blocks: a plugin
+ * inside an inference engine whose enqueue step may not allocate (the
+ * engine owns all device memory and passes in only inputs and outputs),
+ * code between the begin and end of a stream capture (cudaMalloc is not a
+ * stream operation and may synchronise the device), or a process that has
+ * handed all device memory to its own pool allocator.  This call takes the
+ * same inputs and outputs as jattn_sparse_select minus the qbar / kbar
+ * workspace, which lives instead in a fixed 16 MiB device array inside the
+ * library (held by every GPU that loads the library until the process
+ * exits).  It allocates and frees nothing.
+ *
+ * q, k, probs, kv_idx, kv_cnt, sizes, softmax_scale, tau : as for
+ * jattn_sparse_select, with the same results.
+ * Limit: B * H * (ceil(N / 256) + ceil(N / 128)) * 128 * 4 bytes must not
+ * exceed 16 MiB (B = 2, H = 24 up to N = 58112); a larger problem is
+ * rejected with JATTN_ERR_UNSUPPORTED before anything is launched.
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Later calls on the device reuse the address.
+ * Sharing: every call uses the same array and leaves its contents behind.
+ * Each call overwrites every part of it that it reads, so nothing needs to
+ * start at zero, but two calls whose work overlaps on the GPU (on
+ * different streams, or from different threads) race on the array and
+ * give undefined results: serialise them.
+ */
+JATTN_API int jattn_sparse_select_noalloc(const void* q, const void* k, float* probs, int* kv_idx, int* kv_cnt,
+                                int B, int H, int N_txt, int N_img, int N_ref, int d,
+                                float softmax_scale, float tau, void* cuda_stream);
+
 /* Human-readable name of a jattn_status value (static string, never NULL). */
 JATTN_API const char* jattn_status_string(int status);
 
