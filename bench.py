@@ -9,10 +9,19 @@ tokens).  The metric is attention TFLOP/s with FLOPs = 4 * B * H * N^2 * d.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Under torchrun every rank runs its own independent batch (weak scaling, no
-data-path collective); the step time is the max over ranks.  Rank 0 prints
-one JSON line.  ``--impl reference`` times the float64 CPU oracle instead,
-on a bounded sample of the same workload, on rank 0 only.
+The attention's K input carries the workload's outliers: the prologue's K'
+with 1% of its (b, t, h) rows scaled by 8 (RMSNorm would erase an outlier in
+raw K), built once before the timed region.
+
+Under torchrun (N > 1) the ranks split one problem the way the tutorial's
+multi-GPU section does: the two CFG branches (the batch) on separate rank
+groups and Ulysses sequence parallelism inside a group, an all-to-all of Q,
+K, V to head shards before the attention and one of O back after it, over
+NCCL (strong scaling).  ``--replicas`` runs an independent full problem per
+rank instead (weak scaling, no data-path collective).  The step time is the
+max over ranks; rank 0 prints one JSON line.  ``--impl reference`` times the
+float64 CPU oracle instead, on a bounded sample of the same workload, on
+rank 0 only.
 """
 
 from __future__ import annotations
@@ -44,7 +53,7 @@ PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_bf16_traffic_t2i_2048.md"
 KERNEL_SOURCES = ["attn_bf16.cu", "sm100_ptx.cuh", "softmax_sm100.cuh", "jattn_internal.h"]
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
@@ -54,13 +63,17 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU oracle baseline budget (rank 0, N=1)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-table", action="store_true",
+                    help="time the float64 oracle on all five workloads (minutes of host CPU) and exit")
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-path timing object")
     ap.add_argument("--no-qkv", action="store_true", help="skip the fused-QKV-projection timing object")
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse attention timing object")
-    ap.add_argument("--sp", action="store_true",
-                    help="Ulysses sequence parallelism over all ranks (strong scaling of one problem) "
-                         "instead of one independent problem per rank")
-    return ap.parse_args()
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N > 1 ranks: an independent full problem per rank (weak scaling) instead of "
+                         "the CFG x Ulysses split of one problem")
+    ap.add_argument("--cfg", type=int, default=2,
+                    help="CFG degree of the multi-GPU layout (ranks = cfg x sequence-parallel degree)")
+    return ap.parse_args(argv)
 
 
 def workload_config(w: I.Workload, extra=None):
@@ -209,11 +222,80 @@ def cpu_baseline(w: I.Workload, q, k, v, seconds: float):
         done += 1
     dt = time.perf_counter() - t0
     rate = flops / dt / 1e12
-    return {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    return {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "cpu_model": cpu_model(),
+            "cpu_count": os.cpu_count(),
             "sample": (f"float64 oracle (prologue of one (b,h) slice + attention of {rows_per_unit} sampled "
                        f"query rows vs all {w.N} keys) on {done} of {len(units)} (b,h) pairs, {dt:.1f} s"),
             "full_step_s_extrapolated": w.flops / (rate * 1e12),
             "seconds": dt}
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (lscpu, else /proc/cpuinfo)."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.startswith("Model name:"):
+                return line.split(":", 1)[1].strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+CPU_TABLE_CONFIGS = ("tiny", "t2i_1024", "t2i_2048", "i2i_2048", "t2i_2048_fp8")
+
+
+def cpu_baseline_table(rows_sampled: int = 256):
+    """The float64 oracle on every workload, on the host cores: tiny and
+    t2i_1024 in full; the 2048^2 workloads on ``rows_sampled`` sampled query
+    rows per (b, h) against all keys, with the full-size time extrapolated
+    (prologue time + attention time x N / rows).  Every (b, h) is run; the
+    FP8 workload also quantises Q', K', V to E4M3 blocks and dequantises
+    them before the attention.  One JSON object per workload."""
+    import oracle as O
+    out = []
+    for name in CPU_TABLE_CONFIGS:
+        w = I.WORKLOADS[name]
+        q, k, v = I.make_qkv(w, seed=0)
+        full = name in ("tiny", "t2i_1024")
+        rows = None if full else I.sampled_rows(w, rows_sampled)
+        n_rows = w.N if full else len(rows)
+        t_pro = t_att = 0.0
+        for b in range(w.B):
+            for h in range(w.H):
+                t0 = time.perf_counter()
+                qs = q[b:b + 1, :, h:h + 1, :].float().numpy()
+                ks = k[b:b + 1, :, h:h + 1, :].float().numpy()
+                vs = v[b:b + 1, :, h:h + 1, :].float().numpy()
+                qp, kp = O.prologue(qs, ks, n_txt=w.n_txt, img_h=w.img_h, img_w=w.img_w, ref_h=w.ref_h,
+                                    ref_w=w.ref_w, ref_row_offset=w.ref_row_offset, theta=w.theta, eps=w.eps)
+                qp, kp = O.bf16_round(qp), O.bf16_round(kp)
+                if w.path == "fp8":
+                    qp, kp, vs = (O.dequantize_e4m3(*O.block_quantize_e4m3(x)) for x in (qp, kp, vs))
+                t1 = time.perf_counter()
+                O.joint_attention(qp, kp, vs, w.softmax_scale, rows=rows)
+                t2 = time.perf_counter()
+                t_pro += t1 - t0
+                t_att += t2 - t1
+        flops_done = 4.0 * w.B * w.H * n_rows * w.N * w.d
+        full_s = t_pro + t_att * (w.N / n_rows)
+        out.append({
+            "workload": name, "B": w.B, "H": w.H, "N": w.N, "path": w.path,
+            "rows_per_head": n_rows, "sampled": not full,
+            "measured_s": t_pro + t_att, "prologue_s": t_pro, "attention_s": t_att,
+            "attention_gflops": flops_done / t_att / 1e9,
+            "full_step_s": full_s, "full_step_extrapolated": not full,
+            "flops_full": w.flops,
+        })
+    return {"cpu_model": cpu_model(), "cpu_count": os.cpu_count(), "blas_threads": blas_threads(),
+            "kind": "oracle (float64 numpy)", "configs": out}
 
 
 def run_reference(args, rank: int, world: int):
@@ -490,7 +572,30 @@ def weak_scaling_value(world: int, flops_per_rank: float, ms_per_step: float) ->
     return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
-def run_e2e(J, w, q, k, v, dev, params, steps):
+def outlier_k(J, w, qd, kd, params, seed, stream):
+    """The attention's K input of the stated workload: K' = the prologue of
+    K, with the workload's outlier rows (1% of (b, t, h) rows on t2i_2048)
+    scaled by the outlier gain.  RMSNorm would erase an outlier in raw K, so
+    the scaling applies to K'.  Built once, outside the timed region."""
+    qp, kp = torch.empty_like(qd), torch.empty_like(kd)
+    J.jattn_prologue(qd, kd, None, qp, kp, None, None, None, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+                     J.JATTN_PROLOGUE_BF16, params, stream.cuda_stream)
+    torch.cuda.synchronize(qd.device)
+    if w.k_outlier_frac <= 0:
+        return kp
+    mask = I.outlier_rows(w, seed)
+    return I.apply_outliers(kp.cpu(), mask, w.k_outlier_gain).to(qd.device)
+
+
+def e2e_steps(steps: int) -> int:
+    """Steps of the end-to-end leg: at least 10, at most 20."""
+    return max(10, min(steps, 20))
+
+
+def run_e2e(J, w, q, k, v, k_att, dev, params, steps):
+    """The headline step with host buffers: each step copies Q, K, V from
+    pinned host memory, runs the prologue and the attention (on the outlier
+    K' `k_att`, resident like the weights of a layer) and reads O back."""
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     ins = [[torch.empty_like(qh, device=dev) for _ in range(3)] for _ in range(2)]
     mids = [torch.empty_like(qh, device=dev) for _ in range(2)]       # Q', K' (reused per step)
@@ -500,7 +605,7 @@ def run_e2e(J, w, q, k, v, dev, params, steps):
     h2d_done = [torch.cuda.Event() for _ in range(2)]
     comp_done = [torch.cuda.Event() for _ in range(2)]
     d2h_done = [torch.cuda.Event() for _ in range(2)]
-    Ke = max(4, steps // 5)
+    Ke = e2e_steps(steps)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     def issue_h2d(i):
@@ -527,7 +632,7 @@ def run_e2e(J, w, q, k, v, dev, params, steps):
             qp, kp = mids
             J.jattn_prologue(qd, kd, None, qp, kp, None, None, None, None, w.B, w.H, w.n_txt, w.n_img,
                              w.n_ref, w.d, J.JATTN_PROLOGUE_BF16, params, comp)
-            J.jattn_fwd_bf16(qp, kp, vd, outs[bi], None, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
+            J.jattn_fwd_bf16(qp, k_att, vd, outs[bi], None, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d,
                              w.softmax_scale, comp)
             comp_done[bi].record(comp)
         with torch.cuda.stream(d2h):
@@ -541,6 +646,8 @@ def run_e2e(J, w, q, k, v, dev, params, steps):
 
 
 def run_ours(args, rank: int, world: int, local_rank: int):
+    """One full problem per rank: the headline at N = 1, and independent
+    replicas (weak scaling, no data-path collective) with --replicas."""
     from diffusion_transformer_joint_dit_b200 import binding as J
 
     dist = world > 1
@@ -558,14 +665,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     params = J.make_prologue_params(w.img_h, w.img_w, w.ref_h, w.ref_w, w.ref_row_offset, w.theta, w.eps)
     stream = torch.cuda.current_stream(dev)
     s_handle = stream.cuda_stream
+    # The attention's K input carries the workload's outliers (see outlier_k);
+    # plain K' (the prologue's output, no outliers) is timed beside it.
+    k_att = outlier_k(J, w, qd, kd, params, rank, stream)
 
     def prologue():
         J.jattn_prologue(qd, kd, None, qp, kp, None, None, None, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref,
                          w.d, J.JATTN_PROLOGUE_BF16, params, s_handle)
 
-    def attention():
-        J.jattn_fwd_bf16(qp, kp, vd, o, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d, w.softmax_scale,
-                         s_handle)
+    def attention(kin=None):
+        J.jattn_fwd_bf16(qp, k_att if kin is None else kin, vd, o, None, w.B, w.H, w.n_txt, w.n_img, w.n_ref,
+                         w.d, w.softmax_scale, s_handle)
 
     for _ in range(max(args.warmup, 3)):
         prologue()
@@ -605,6 +715,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     pro_med = statistics.median(a.elapsed_time(b) for a, b in pro_ev)
     if J.jattn_device_status(s_handle) != J.JATTN_OK:
         raise RuntimeError("device error word set during timed steps")
+    # The same attention on plain K' (no outliers), for comparison.
+    plain_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(min(K, 20))]
+    for a, b in plain_ev:
+        a.record(stream)
+        attention(kp)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    att_plain = statistics.mean(a.elapsed_time(b) for a, b in plain_ev)
 
     # ---- end-to-end region: host buffers, copies inside the timed region ----
     # Every step copies its Q, K, V from pinned host memory and reads its O
@@ -613,9 +732,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # and outputs double-buffered).  Timed from the first copy to the last.
     if dist:
         torch.distributed.barrier()
-    e2e_elapsed, Ke = run_e2e(J, w, q, k, v, dev, params, K)
-    elapsed, e2e_elapsed, att_ms, pro_ms, att_med, pro_med = max_over_ranks(
-        [elapsed, e2e_elapsed, att_ms, pro_ms, att_med, pro_med], dev)
+    e2e_elapsed, Ke = run_e2e(J, w, q, k, v, k_att, dev, params, K)
+    elapsed, e2e_elapsed, att_ms, pro_ms, att_med, pro_med, att_plain = max_over_ranks(
+        [elapsed, e2e_elapsed, att_ms, pro_ms, att_med, pro_med, att_plain], dev)
     if dist:
         torch.distributed.destroy_process_group()
     if rank != 0:
@@ -630,17 +749,25 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     achieved = w.flops / (att_ms * 1e-3) / 1e12
     traffic = profiled_traffic()
     act_bytes = w.B * w.N * w.H * w.d * 2
+    data = "synthetic (seeded N(0,1) bf16 Q, K, V"
+    if w.k_outlier_frac > 0:
+        data += (f"; the attention's K input is the prologue's K' with {w.k_outlier_frac:.0%} of (b, t, h) rows "
+                 f"x{w.k_outlier_gain:g}")
+    data += ")"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q, K, V; random-free kernels)",
+        "dtype": "bf16", "data": data,
         "config": workload_config(w, {"attention_ms": att_ms, "prologue_ms": pro_ms,
                                       "attention_ms_median": att_med, "prologue_ms_median": pro_med,
+                                      "attention_ms_plain_k": att_plain,
+                                      "attention_tflops_plain_k": w.flops / (att_plain * 1e-3) / 1e12,
                                       "prologue_gbs": 4 * act_bytes / (pro_ms * 1e-3) / 1e9}),
         "roofline": {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": traffic,
             "kernel": "attn_bf16_kernel", "flops_per_launch": w.flops,
+            "data": "outlier K'" if w.k_outlier_frac > 0 else "plain",
             "peak_source": f"{peaks_src} {'bf16_tflops_sustained' if sustained else 'bf16_tflops'}"
                            f" ({'timed region >= 1 s' if sustained else 'timed region < 1 s'})",
             "algorithmic_bytes_per_launch": 4 * act_bytes,
@@ -656,6 +783,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "gpu_launches": 2 * K,
         "clocks": clocks,
     }
+    if world > 1:
+        line["config"]["parallelism"] = f"replicas: an independent {w.name} problem per GPU (no collective)"
     if not args.no_fp8:
         line["fp8_path"] = time_fp8_path(J, dev, stream, rank, peaks, peaks_src)
     if not args.no_qkv:
@@ -669,32 +798,80 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return 0
 
 
-def run_sp(args, rank: int, world: int, local_rank: int):
-    """One problem split over all ranks by Ulysses sequence parallelism: each
-    rank holds its sequence shard of Q, K, V in HBM; a step is the exchange
-    to head shards, the prologue and BF16 attention on H / P heads, and the
-    exchange back.  Total work is fixed as ranks are added (strong scaling)."""
+# ---------------------------------------------------- CFG x Ulysses (N > 1) --
+
+def cfg_ulysses_plan(w: I.Workload, world: int, rank: int, cfg: int):
+    """This rank's share of one problem under the tutorial's multi-GPU
+    layout: the CFG branches (the batch) split over ``cfg`` rank groups, and
+    inside a group the joint sequence split over the ``world / cfg`` ranks
+    (Ulysses).  Returns (layout, batch slice, sequence shard [s0, s1))."""
+    from diffusion_transformer_joint_dit_b200 import ulysses as U
+
+    if cfg < 1 or w.B % cfg != 0 or world % cfg != 0:
+        cfg = 1
+    layout = U.ParallelLayout.make(world, cfg)
+    if w.H % layout.sp != 0:
+        raise SystemExit(f"{w.H} heads do not split over {layout.sp} sequence ranks")
+    per = w.B // layout.cfg
+    c = layout.cfg_index(rank)
+    s0, s1 = U.shard_bounds(w.N, layout.sp, layout.sp_rank(rank))
+    return layout, slice(c * per, (c + 1) * per), (s0, s1)
+
+
+def cfg_ulysses_step(q, k, v, k_att_heads, n_total, prologue, attn, group=None):
+    """One step of a rank: exchange its sequence shard of Q, K, V to the head
+    shard of the whole sequence, the prologue there (positions are global),
+    attention with the head shard's K input ``k_att_heads`` (the prologue's
+    K' carrying the workload's outliers), and O back to the sequence shard."""
+    from diffusion_transformer_joint_dit_b200 import ulysses as U
+
+    p = torch.distributed.get_world_size(group)
+    if p == 1:  # the whole sequence is here: no exchange
+        qp, _, vp = prologue(q, k, v)
+        return attn(qp, k_att_heads, vp)
+    sizes = U.shard_sizes(n_total, p)
+    qh, kh, vh = (U.seq_to_heads(t, sizes, group) for t in (q, k, v))
+    qp, _, vh = prologue(qh, kh, vh)
+    return U.heads_to_seq(attn(qp, k_att_heads, vh), sizes, group)
+
+
+def run_cfg_ulysses(args, rank: int, world: int, local_rank: int):
+    """One problem split over all ranks (strong scaling): the CFG branches on
+    separate rank groups (no exchange between them) and Ulysses sequence
+    parallelism inside a group (one all-to-all before the attention, one
+    after, over NCCL).  Every rank holds its shard of Q, K, V in HBM."""
     from diffusion_transformer_joint_dit_b200 import binding as J
     from diffusion_transformer_joint_dit_b200 import ulysses as U
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-    os.environ.setdefault("MASTER_PORT", "29531")
-    torch.distributed.init_process_group("nccl", rank=rank, world_size=world,
-                                         timeout=datetime.timedelta(seconds=120), device_id=dev)
+    torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    group = None
     try:
         w = I.WORKLOADS[args.workload]
-        if w.path != "bf16" or w.H % world != 0:
-            raise SystemExit("--sp needs a BF16 workload whose heads split over the ranks")
+        if w.path != "bf16":
+            raise SystemExit("bench.py times the BF16 path")
+        layout, bsl, (s0, s1) = cfg_ulysses_plan(w, world, rank, args.cfg)
+        group = U.new_sp_groups(layout)
         q, k, v = I.make_qkv(w, seed=0)
-        s0, s1 = U.shard_bounds(w.N, world, rank)
-        qd, kd, vd = (t[:, s0:s1].contiguous().to(dev) for t in (q, k, v))
+        qd, kd, vd = (t[bsl, s0:s1].contiguous().to(dev) for t in (q, k, v))
+        nb = bsl.stop - bsl.start
+        hp = w.H // layout.sp
+        me = layout.sp_rank(rank)
         prologue, attn = U.jattn_bf16_ops(w.n_txt, w.n_img, w.n_ref, w.softmax_scale, w.img_h, w.img_w,
                                           w.ref_h, w.ref_w, w.ref_row_offset)
+        # The head shard's attention K input: its K' with the workload's
+        # outlier rows (the same (b, t, h) rows as on one GPU), built once.
+        sizes = U.shard_sizes(w.N, layout.sp)
+        qh, kh, vh = (U.seq_to_heads(t, sizes, group) for t in (qd, kd, vd))
+        _, kph, _ = prologue(qh, kh, vh)
+        if w.k_outlier_frac > 0:
+            mask = I.outlier_rows(w, 0)[bsl, :, me * hp:(me + 1) * hp]
+            kph = I.apply_outliers(kph.cpu(), mask.copy(), w.k_outlier_gain).to(dev)
+        del qh, kh, vh
 
         def step():
-            return U.ulysses_attention(qd, kd, vd, n_total=w.N, attn=attn, prologue=prologue)
+            return cfg_ulysses_step(qd, kd, vd, kph, w.N, prologue, attn, group)
 
         for _ in range(max(args.warmup, 3)):
             step()
@@ -707,6 +884,7 @@ def run_sp(args, rank: int, world: int, local_rank: int):
         torch.distributed.barrier()
         torch.cuda.synchronize(dev)
         clocks.start()
+        time.sleep(0.3)
         e0.record()
         for _ in range(K):
             step()
@@ -720,14 +898,19 @@ def run_sp(args, rank: int, world: int, local_rank: int):
         if rank == 0:
             value = w.flops / (ms * 1e-3) / 1e12
             line = {
-                "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+                "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
                 "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
                 "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
-                "data": "synthetic (seeded N(0,1) bf16 Q, K, V)",
+                "data": "synthetic (seeded N(0,1) bf16 Q, K, V; the attention's K input is the prologue's K' "
+                        f"with {w.k_outlier_frac:.0%} of (b, t, h) rows x{w.k_outlier_gain:g})",
                 "config": workload_config(w, {
-                    "path": "bf16", "parallelism": f"ulysses sp{world} (all-to-all over NCCL)",
-                    "step": "all-to-all to head shards + jattn_prologue + jattn_fwd_bf16 on H/P heads + "
-                            "all-to-all back",
+                    "parallelism": f"cfg{layout.cfg} x ulysses sp{layout.sp} (all-to-all over NCCL inside a "
+                                   f"CFG group; no exchange between groups)",
+                    "step": "all-to-all of Q, K, V to head shards + jattn_prologue + jattn_fwd_bf16 on "
+                            f"H/{layout.sp} heads + all-to-all of O back",
+                    "per_rank": f"batch {bsl.start}..{bsl.stop - 1}, tokens {s0}..{s1 - 1} of {w.N}",
+                    "all_to_all_bytes_sent_per_rank_per_step":
+                        4 * nb * (s1 - s0) * w.H * w.d * 2 * (layout.sp - 1) // layout.sp,
                     "l2": "inputs larger than L2"}),
                 "gpu_launches": 2 * K,
                 "clocks": clk,
@@ -745,10 +928,14 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         raise SystemExit("--gpus N > 1 runs under torchrun (one process per GPU)")
+    if args.cpu_table:
+        if rank == 0:
+            print(json.dumps(cpu_baseline_table()), flush=True)
+        return 0
     if args.impl == "reference":
         return run_reference(args, rank, world)
-    if args.sp:
-        return run_sp(args, rank, world, local_rank)
+    if world > 1 and not args.replicas:
+        return run_cfg_ulysses(args, rank, world, local_rank)
     return run_ours(args, rank, world, local_rank)
 
 

@@ -50,8 +50,40 @@ def joint_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, n_txt:
     cfg = config or AttentionConfig()
     if cfg.mode not in MODES:
         raise ValueError(f"mode must be one of {MODES}")
-    if q.dtype != torch.bfloat16 or not q.is_cuda:
-        raise ValueError("q, k, v must be bf16 CUDA tensors")
+    q, k, v = _checked_inputs(q, k, v)
+    q_norm_w, k_norm_w = (_checked_weight(w_, q) for w_ in (q_norm_w, k_norm_w))
+    with torch.cuda.device(q.device):
+        return _joint_attention(q, k, v, n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset, ref_grids, cfg,
+                                softmax_scale, q_norm_w, k_norm_w, return_lse)
+
+
+def _checked_inputs(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
+    """q, k, v as the library needs them: bf16 CUDA tensors of one shape
+    [B, N, H, d] on one device, contiguous (a strided view, e.g. from
+    qkv.unbind(2), is copied)."""
+    ts = (q, k, v)
+    if any(not isinstance(t, torch.Tensor) for t in ts):
+        raise TypeError("q, k, v must be torch tensors")
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError(f"q, k, v must share one [B, N, H, d] shape, got {tuple(q.shape)}, {tuple(k.shape)}, "
+                         f"{tuple(v.shape)}")
+    if any(t.dtype != torch.bfloat16 for t in ts):
+        raise ValueError("q, k, v must be bf16")
+    if any(not t.is_cuda for t in ts) or k.device != q.device or v.device != q.device:
+        raise ValueError("q, k, v must be CUDA tensors on one device")
+    return tuple(t.contiguous() for t in ts)
+
+
+def _checked_weight(w_, q: torch.Tensor):
+    if w_ is None:
+        return None
+    if w_.dtype != torch.float32 or w_.shape != (q.shape[-1],) or w_.device != q.device:
+        raise ValueError("norm weights must be fp32 [d] tensors on q's device")
+    return w_.contiguous()
+
+
+def _joint_attention(q, k, v, n_txt, img_h, img_w, ref_h, ref_w, ref_row_offset, ref_grids, cfg, softmax_scale,
+                     q_norm_w, k_norm_w, return_lse):
     B, N, H, d = q.shape
     n_img = img_h * img_w
     n_ref = N - n_txt - n_img

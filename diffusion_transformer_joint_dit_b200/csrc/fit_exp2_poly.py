@@ -8,7 +8,7 @@ started from Chebyshev nodes.  The softmax stores P in bf16 (8 significant
 bits) or fp16 (11 bits), so a relative error near 2^-13 is ample.
 
 Run:  python fit_exp2_poly.py   (prints the coefficients and the error)
-The printed float32 coefficients are the ones in attn_bf16.cu.
+The printed float32 coefficients are kPolyC0..kPolyC3 in softmax_sm100.cuh.
 """
 
 import numpy as np

@@ -138,13 +138,18 @@ int fill_positions(PrologueArgs& a, const jattn_prologue_params* p, int N_txt, i
 }  // namespace
 
 cudaError_t make_act_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int elem_bytes) {
+  return make_act_map_box(map, ptr, B, N, H, elem_bytes, 128);
+}
+
+cudaError_t make_act_map_box(CUtensorMap* map, const void* ptr, int B, int N, int H, int elem_bytes,
+                             int box_tokens) {
   EncodeTiledFn fn = encoder();
   if (fn == nullptr) return cudaErrorNotSupported;
   const cuuint64_t row = static_cast<cuuint64_t>(kHeadDim) * elem_bytes;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {row, row * H, row * H * N};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 1, 128, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), 1, static_cast<cuuint32_t>(box_tokens), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUresult r = fn(map, dt, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,

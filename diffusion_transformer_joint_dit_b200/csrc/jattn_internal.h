@@ -126,6 +126,10 @@ cudaError_t launch_wait_selftest(uint64_t timeout_ns, cudaStream_t s);
 // up via the runtime's driver entry point (no link-time libcuda dependency).
 cudaError_t make_act_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int elem_bytes);
 
+// The same view with a box of `box_tokens` tokens (1 .. 256) instead of 128.
+cudaError_t make_act_map_box(CUtensorMap* map, const void* ptr, int B, int N, int H, int elem_bytes,
+                             int box_tokens);
+
 // 4-D tensor map over a token-major bf16 [B, N, H, d=128] tensor for the
 // prologue: box (128 channels, `box_heads` heads, `box_tokens` tokens, 1),
 // no swizzle (rows land densely, 256 B each, token-major then head), zero

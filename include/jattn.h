@@ -347,7 +347,8 @@ JATTN_API int jattn_sparse_select(const void* q, const void* k, float* qbar, flo
  * The list must be strictly increasing key-block indices in [0, n_kb);
  * counts are clamped to [0, n_kb] and indices into [0, n_kb) so that any
  * list stays within the tensors, but a list that breaks the rule gives
- * undefined values.
+ * undefined values (a repeated index, for one, counts its keys twice in O
+ * and the LSE).  Nothing checks the rule at run time.
  */
 JATTN_API int jattn_fwd_bf16_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
                           const int* kv_idx, const int* kv_cnt,
@@ -402,7 +403,13 @@ JATTN_API const char* jattn_last_cuda_error(void);
  * jattn_device_status — synchronise `cuda_stream`, read and clear the device
  * error word the kernels set when a bounded wait runs out.  Returns JATTN_OK,
  * JATTN_ERR_TIMEOUT, or JATTN_ERR_CUDA if the synchronisation itself failed.
- * A diagnostic call: it blocks the host and must not be stream-captured.
+ * The error word is one per device and process: it collects timeouts of
+ * every launch of the library on the current device since the last call,
+ * from any stream or host thread, and this call clears it for all of them.
+ * Synchronising `cuda_stream` only waits for that stream's work; a timeout
+ * in a launch still running on another stream may be reported by a later
+ * call.  A diagnostic call: it blocks the host and must not be
+ * stream-captured.
  */
 JATTN_API int jattn_device_status(void* cuda_stream);
 

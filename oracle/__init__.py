@@ -24,8 +24,8 @@ arithmetic.  Sources (titles of the web pages the method is described on):
 
 The pages fix no constants (head size, eps, RoPE base and axis split, block
 size, quantisation format); those come from the workload definitions and
-the readings listed in the design notes, each repeated in the docstring of
-the function that applies it.
+from readings of the pages, each stated in the docstring of the function
+that applies it.
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py``
 against closed forms, hand-derived worked values (``tests/golden/``),

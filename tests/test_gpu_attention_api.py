@@ -55,3 +55,16 @@ def test_sparse_mode_at_tau_zero_is_the_bf16_mode(cuda_ok):
     o_dense, l_dense = _call("bf16", q, k, v)
     o_sparse, l_sparse = _call("sparse", q, k, v, tau=0.0)
     assert torch.equal(o_dense, o_sparse) and torch.equal(l_dense, l_sparse)
+
+
+def test_strided_views_give_the_contiguous_result(cuda_ok):
+    """q, k, v as views of one packed [B, N, 3, H, d] projection output (not
+    contiguous) give the same result as contiguous copies."""
+    q, k, v = I.make_qkv(W, seed=24)
+    packed = torch.stack([q, k, v], dim=2).cuda()
+    qv, kv, vv = packed.unbind(2)
+    assert not qv.is_contiguous()
+    o_view, l_view = A.joint_attention(qv, kv, vv, n_txt=W.n_txt, img_h=W.img_h, img_w=W.img_w, ref_h=W.ref_h,
+                                       ref_w=W.ref_w, ref_row_offset=W.ref_row_offset, return_lse=True)
+    o, lse = _call("bf16", q, k, v)
+    assert torch.equal(o_view, o) and torch.equal(l_view, lse)

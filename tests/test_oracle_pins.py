@@ -376,7 +376,7 @@ def test_inputs_are_seeded_and_shaped():
 
 
 # ---------------------------------------------------------------------------
-# RoPE table and the fused QKV projection (NEXT-2)
+# RoPE table and the fused QKV projection
 # ---------------------------------------------------------------------------
 
 def test_rope_table_closed_form_entries():
@@ -463,7 +463,7 @@ def test_qkv_fused_value_brute_force_and_norm_weights():
 
 
 # ---------------------------------------------------------------------------
-# FP8 repair budget (NEXT-3)
+# FP8 repair budget
 # ---------------------------------------------------------------------------
 
 def test_repair_count():
