@@ -26,11 +26,17 @@
 // rescale O_i and overwrite P_i.
 //
 // Online softmax in the exp2 domain with a lazy maximum: the reference max
-// m of a row only moves when the new tile's max exceeds it by more than 8
-// (log2 units); P is then at most 2^8, harmless for bf16 P and fp32 O / l.
+// m of a row only moves when the new tile's max exceeds it by more than 16
+// (log2 units); P is then at most 2^16, harmless for bf16 P and fp32 O / l.
 // The O rescale (a TMEM read-modify-write) is thus rare after the first
-// tiles.  Tail keys (N not a multiple of 128) are masked to -inf; tail
-// query rows read zero-filled Q and are not stored.
+// tiles, keys with outlier logits included.  Tail keys (N not a multiple of
+// 128) are masked to -inf; tail query rows read zero-filled Q and are not
+// stored.
+//
+// The row sum is formed after P is handed to the MMA issuer, off the path
+// to the next P.V.  The producer and MMA threads wait with suspending
+// mbarrier waits, so that they take no issue slots from the softmax warps
+// of their SM sub-partitions while they wait.
 //
 // Block-sparse variant (kSparse): the tutorial's Sol-Attention runs a
 // generic block-sparse attention kernel.  A CTA's 256 query rows are one
@@ -58,12 +64,7 @@ constexpr int kLoadWarp = kSoftmaxWarps;       // 8
 constexpr int kMmaWarp = kSoftmaxWarps + 1;    // 9
 constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;
-// Share of exp2 pairs sent to the polynomial (0 = all on MUFU).  Measured
-// on B200 at 2048^2: all-MUFU is fastest at this kernel's 168-register
-// budget (10 warps, three on one SM sub-partition); 1 in 4 is ~9% slower
-// and 1 in 2 spills.
-constexpr int kPolyEvery = 0;
+constexpr float kRescaleThreshold = 16.0f;
 
 struct Ctrl {
   uint64_t q_full;
@@ -95,7 +96,7 @@ struct Params {
 // Wait that only gives up on time (used while draining at teardown).
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
   int never = 0;
-  return mbar_wait(bar, parity, &never, timeout_ns);
+  return mbar_wait_sleep(bar, parity, &never, timeout_ns);
 }
 
 template <bool kSparse>
@@ -171,7 +172,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int which = 0; which < 2; ++which, ++it) {
           const int slot = it % kStages;
           const uint32_t round = static_cast<uint32_t>(it / kStages);
-          if (!mbar_wait(&ctrl->kv_empty[slot], (round & 1u) ^ 1u, abort_flag, prm.timeout_ns)) {
+          if (!mbar_wait_sleep(&ctrl->kv_empty[slot], (round & 1u) ^ 1u, abort_flag, prm.timeout_ns)) {
             ok = false;
             break;
           }
@@ -195,34 +196,37 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(1, 1, false, kBM, kBN);  // bf16 x bf16, K-major both
       constexpr uint32_t idesc_pv = make_idesc(1, 1, true, kBM, kD);    // P (TMEM) x V (MN-major)
-      const uint32_t q_base = smem_u32(smem + kSmemQ);
-      const uint32_t ring = smem_u32(smem + kSmemRing);
+      // Descriptors of the first Q tile and ring slot; the start-address
+      // field is bits [0,14) in 16-byte units, so adding (offset >> 4)
+      // moves a descriptor within shared memory.
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + kSmemQ), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(smem + kSmemRing), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(smem + kSmemRing), kBoxBytes, 1024);
 
       auto issue_qk = [&](int t, int slot) {
         const uint32_t d = tmem + t * kBN;  // S_t
-        const uint32_t qa = q_base + t * kTileBytes;
-        const uint32_t kb = ring + slot * kTileBytes;
+        const uint64_t qa = dq0 + static_cast<uint64_t>((t * kTileBytes) >> 4);
+        const uint64_t kb = dk0 + static_cast<uint64_t>((slot * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_f16_ss(d, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024), idesc_qk,
-                     kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4);
+          mma_f16_ss(d, qa + off, kb + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
         const uint32_t d = tmem + 2 * kBN + t * kD;  // O_t
         const uint32_t p = tmem + t * kBN;           // P_t (packed bf16 in S_t columns)
-        const uint32_t vb = ring + slot * kTileBytes;
+        const uint64_t vb = dv0 + static_cast<uint64_t>((slot * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          mma_f16_ts(d, p + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, kBoxBytes, 1024), idesc_pv,
+          mma_f16_ts(d, p + kk * 8, vb + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
                      (acc || kk > 0) ? 1u : 0u);
         }
       };
 
-      bool ok = mbar_wait(&ctrl->q_full, 0, abort_flag, prm.timeout_ns);
+      bool ok = mbar_wait_sleep(&ctrl->q_full, 0, abort_flag, prm.timeout_ns);
       int it = 0;
-      if (ok && n_iter > 0) ok = mbar_wait(&ctrl->kv_full[0], 0, abort_flag, prm.timeout_ns);
+      if (ok && n_iter > 0) ok = mbar_wait_sleep(&ctrl->kv_full[0], 0, abort_flag, prm.timeout_ns);
       if (ok && n_iter > 0) {
         tc_fence_after();
         issue_qk(0, 0);
@@ -234,19 +238,19 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       for (int j = 0; j < n_iter && ok; ++j) {
         const int slot_v = it % kStages;
-        ok = mbar_wait(&ctrl->kv_full[slot_v], static_cast<uint32_t>(it / kStages) & 1u, abort_flag,
+        ok = mbar_wait_sleep(&ctrl->kv_full[slot_v], static_cast<uint32_t>(it / kStages) & 1u, abort_flag,
                        prm.timeout_ns);
         ++it;
         if (!ok) break;
         const bool has_next = j + 1 < n_iter;
         const int slot_k = it % kStages;
         // Q tile 0
-        ok = mbar_wait(&ctrl->p_full[0], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns);
+        ok = mbar_wait_sleep(&ctrl->p_full[0], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns);
         if (!ok) break;
         tc_fence_after();
         issue_pv(0, slot_v, j > 0);
         if (has_next) {
-          ok = mbar_wait(&ctrl->kv_full[slot_k], static_cast<uint32_t>(it / kStages) & 1u, abort_flag,
+          ok = mbar_wait_sleep(&ctrl->kv_full[slot_k], static_cast<uint32_t>(it / kStages) & 1u, abort_flag,
                          prm.timeout_ns);
           if (!ok) break;
           tc_fence_after();
@@ -254,7 +258,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           mma_commit(&ctrl->s_full[0]);
         }
         // Q tile 1
-        ok = mbar_wait(&ctrl->p_full[1], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns);
+        ok = mbar_wait_sleep(&ctrl->p_full[1], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns);
         if (!ok) break;
         tc_fence_after();
         issue_pv(1, slot_v, j > 0);
@@ -320,27 +324,27 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       // P = exp2(s * scale * log2e - m), packed two bf16 per 32-bit word in
       // place: keys [0,64) land in sv[0], keys [64,128) in sv[2].
-      float l0, l1;
-      exp_pack_tile<false, kPolyEvery, true>(sv, sl2, -m, sl2, -m, nvalid >= kBN, l0, l1);
-      l += l0 + l1;
+      exp_pack_only<false>(sv, sl2, -m, sl2, -m);
       tmem_st32(s_addr, sv[0]);
       tmem_st32(s_addr + 32, sv[2]);
       // O correction after P is out of registers (keeps register pressure
       // down); it only has to land before this tile's P.V is issued.
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(o_addr + c * 32, ov);
-          tmem_ld_wait(ov);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t ov[16];
+          tmem_ld16(o_addr + c * 16, ov);
+          tmem_ld_wait16(ov);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-          tmem_st32(o_addr + c * 32, ov);
+          for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+          tmem_st16(o_addr + c * 16, ov);
         }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctrl->p_full[t]);
+      // Row sum of the rounded P, after the hand-off.
+      l += sum_packed<false>(sv[0]) + sum_packed<false>(sv[2]);
     }
 
     if (ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->o_full, 0, abort_flag, prm.timeout_ns))) {

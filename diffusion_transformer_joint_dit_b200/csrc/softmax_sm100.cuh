@@ -146,4 +146,46 @@ __device__ __forceinline__ void exp_pack_tile(uint32_t (&sv)[4][32], float c_lo,
   sum_hi = f2_lo(acc_hi) + f2_hi(acc_hi);
 }
 
+// P = exp2(s * c + b) of a 128-key tile with (c, b) per 64-key half,
+// packed in place two per word (keys [0,64) into sv[0], [64,128) into
+// sv[2]) as bf16 or fp16; no row sum (see sum_packed).
+template <bool kF16>
+__device__ __forceinline__ void exp_pack_only(uint32_t (&sv)[4][32], float c_lo, float b_lo, float c_hi, float b_hi) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float cc = c < 2 ? c_lo : c_hi;
+    const float bb = c < 2 ? b_lo : b_hi;
+    const uint64_t cc2 = f2_pack(cc, cc), bb2 = f2_pack(bb, bb);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1])), cc2, bb2);
+      const float lo = ex2_approx(f2_lo(x)), hi = ex2_approx(f2_hi(x));
+      sv[c & 2][(c & 1) * 16 + (i >> 1)] = kF16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
+    }
+  }
+}
+
+// fp32 sum of the 64 bf16 (kF16 = false) or fp16 values packed two per
+// word in p[0..31]: the P values exactly as the P.V MMA multiplies V by
+// them, so that the row sum and the numerator use one set of weights.
+template <bool kF16>
+__device__ __forceinline__ float sum_packed(const uint32_t (&p)[32]) {
+  float a = 0.f, b = 0.f, c = 0.f, d = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    if (kF16) {
+      const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&p[i]));
+      const float2 y = __half22float2(*reinterpret_cast<const __half2*>(&p[i + 1]));
+      a += x.x; b += x.y; c += y.x; d += y.y;
+    } else {
+      asm("{\n\t.reg .b16 l0, h0, l1, h1;\n\tmov.b32 {l0, h0}, %4;\n\tmov.b32 {l1, h1}, %5;\n\t"
+          "add.rn.f32.bf16 %0, l0, %0;\n\tadd.rn.f32.bf16 %1, h0, %1;\n\t"
+          "add.rn.f32.bf16 %2, l1, %2;\n\tadd.rn.f32.bf16 %3, h1, %3;\n\t}"
+          : "+f"(a), "+f"(b), "+f"(c), "+f"(d)
+          : "r"(p[i]), "r"(p[i + 1]));
+    }
+  }
+  return (a + b) + (c + d);
+}
+
 }  // namespace jattn
