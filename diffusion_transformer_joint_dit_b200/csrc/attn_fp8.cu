@@ -7,15 +7,19 @@
 //
 //   S_raw = q8 . k8 on the tensor core (tcgen05 kind::f8f6f4, fp32 accum);
 //   x     = S_raw * (sq(row) * sk(col block) * softmax_scale * log2 e);
-//   P'    = exp2(x - m + log2(sv(col block) / 2^e)), written to TMEM as FP16;
-//   O    += P' . V16 with V16 the E4M3 codes widened to FP16 (exact);
-//   l     = sum over blocks of (sum P') * 2^e / sv(block);
+//   P     = exp2(x - m), written to TMEM as FP16;
+//   V16   = code * (sv(block) / 2^e), widened and scaled to FP16 in shared
+//           memory by the converter warps;
+//   O    += P . V16;  l = sum P (the FP16 values the MMA uses);
 //   O     = O * 2^e / l.
 //
-// The V block scale rides in the exponent bias of the exp2 argument, so it
-// costs the softmax nothing; 2^e >= max_block sv(b, h) keeps P' <= 2^8.  P
-// is FP16 (not E4M3): an E4M3 P costs about 2.5% relative L2, FP16 P about
-// 2e-4 on these workloads.
+// The per-(b, h) power of two 2^e >= max_block sv / 128 keeps |V16| <=
+// 448 * 128 < 65504.  An all-zero V block (scale 1, zero codes) adds
+// nothing to O whatever its factor, and blocks whose scales lie 2^12 below
+// the largest still land in FP16's normal range.  P is FP16 (not E4M3): an
+// E4M3 P costs about 2.5% relative L2, FP16 P about 2e-4 on these
+// workloads.  The lazy maximum moves only when a tile's max exceeds it by
+// more than 14 (log2 units), so P <= 2^14 stays well inside FP16.
 //
 // CTA = 256 query rows of one (b, h) as two 128-row Q tiles, as in the BF16
 // kernel.  Warps: 0-7 softmax (two warpgroups), 8 TMA producer, 9 MMA issuer
@@ -47,11 +51,7 @@ constexpr int kCvtWarp0 = kSoftmaxWarps + 2;   // 10, 11
 constexpr int kCvtThreads = 64;
 constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // 384
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;
-// All exponentials on MUFU: on B200 a 1-in-4 or 1-in-8 polynomial share
-// measured slower (the polynomial's issue slots cost more than the MUFU
-// time it frees at this kernel's register budget).
-constexpr int kPolyEvery = 0;
+constexpr float kRescaleThreshold = 14.0f;
 
 struct Ctrl {
   uint64_t q_full;
@@ -68,8 +68,7 @@ struct Ctrl {
   uint64_t norm_ready;
   uint32_t tmem_base;
   int abort;
-  float v_norm;        // 2^e >= max sv over the (b, h)
-  float v_log2_norm;   // e
+  float v_norm;        // 2^e >= max sv over the (b, h) / 128
 };
 
 constexpr int kSmemQ = 0;
@@ -92,23 +91,26 @@ struct Params {
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
   int never = 0;
-  return mbar_wait(bar, parity, &never, timeout_ns);
+  return mbar_wait_sleep(bar, parity, &never, timeout_ns);
 }
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// 16 E4M3 codes -> 16 FP16 values (exact), as two 16-byte chunks.
-__device__ __forceinline__ void widen16(const uint4& src, uint4& lo, uint4& hi) {
+// 16 E4M3 codes -> 16 FP16 values times the block factor f (an FP16 pair
+// (f, f)), as two 16-byte chunks: each code widens exactly, the product
+// rounds once.
+__device__ __forceinline__ void widen16_scaled(const uint4& src, __half2 f, uint4& lo, uint4& hi) {
   const uint32_t w[4] = {src.x, src.y, src.z, src.w};
   uint32_t out[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] & 0xFFFFu), __NV_E4M3);
     const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[i] >> 16), __NV_E4M3);
-    out[2 * i] = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
-    out[2 * i + 1] = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
+    const __half2 ha = __hmul2(__half2(a), f), hb = __hmul2(__half2(b), f);
+    out[2 * i] = *reinterpret_cast<const uint32_t*>(&ha);
+    out[2 * i + 1] = *reinterpret_cast<const uint32_t*>(&hb);
   }
   lo = make_uint4(out[0], out[1], out[2], out[3]);
   hi = make_uint4(out[4], out[5], out[6], out[7]);
@@ -176,11 +178,11 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int nk = 0, nv = 0;  // fills issued
       for (int j = 0; j < n_kv; ++j) {
         const int ks = j % kKStages, vs = j % kVStages;
-        if (!mbar_wait(&ctrl->k_empty[ks], ((j / kKStages) & 1) ^ 1, abort_flag, prm.timeout_ns)) break;
+        if (!mbar_wait_sleep(&ctrl->k_empty[ks], ((j / kKStages) & 1) ^ 1, abort_flag, prm.timeout_ns)) break;
         mbar_arrive_expect_tx(&ctrl->k_full[ks], kTile8);
         tma_load_4d(smem + kSmemK + ks * kTile8, &tm_k, &ctrl->k_full[ks], 0, h, j * kBN, b);
         ++nk;
-        if (!mbar_wait(&ctrl->v_empty[vs], ((j / kVStages) & 1) ^ 1, abort_flag, prm.timeout_ns)) break;
+        if (!mbar_wait_sleep(&ctrl->v_empty[vs], ((j / kVStages) & 1) ^ 1, abort_flag, prm.timeout_ns)) break;
         mbar_arrive_expect_tx(&ctrl->v_full[vs], kTile8);
         tma_load_4d(smem + kSmemV + vs * kTile8, &tm_v, &ctrl->v_full[vs], 0, h, j * kBN, b);
         ++nv;
@@ -198,32 +200,34 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(0, 0, false, kBM, kBN);  // e4m3 x e4m3, K-major both
       constexpr uint32_t idesc_pv = make_idesc(0, 0, true, kBM, kD);    // f16 P (TMEM) x f16 V (MN-major)
-      const uint32_t q_base = smem_u32(smem + kSmemQ);
-      const uint32_t k_base = smem_u32(smem + kSmemK);
-      const uint32_t vh_base = smem_u32(smem + kSmemVh);
+      // Descriptors of the first tile of each operand; adding (offset >> 4)
+      // to the start-address field moves a descriptor in shared memory.
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + kSmemQ), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(smem + kSmemK), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(smem + kSmemVh), kBox16, 1024);
 
       auto issue_qk = [&](int t, int ks) {
         const uint32_t d = tmem + t * kBN;
-        const uint32_t qa = q_base + t * kTile8;
-        const uint32_t kb = k_base + ks * kTile8;
+        const uint64_t qa = dq0 + static_cast<uint64_t>((t * kTile8) >> 4);
+        const uint64_t kb = dk0 + static_cast<uint64_t>((ks * kTile8) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kD / 32; ++kk) {  // 32 e4m3 channels (32 bytes) per MMA
-          mma_f8_ss(d, smem_desc_sw128(qa + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 32, 16, 1024), idesc_qk,
-                    kk > 0 ? 1u : 0u);
+          mma_f8_ss(d, qa + static_cast<uint64_t>((kk * 32) >> 4), kb + static_cast<uint64_t>((kk * 32) >> 4),
+                    idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int vb, bool acc) {
         const uint32_t d = tmem + 2 * kBN + t * kD;
         const uint32_t p = tmem + t * kBN;
-        const uint32_t v = vh_base + vb * kTile16;
+        const uint64_t v = dv0 + static_cast<uint64_t>((vb * kTile16) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_f16_ts(d, p + kk * 8, smem_desc_sw128(v + kk * 16 * 128, kBox16, 1024), idesc_pv,
+          mma_f16_ts(d, p + kk * 8, v + static_cast<uint64_t>((kk * 16 * 128) >> 4), idesc_pv,
                      (acc || kk > 0) ? 1u : 0u);
       };
 
-      bool ok = mbar_wait(&ctrl->q_full, 0, abort_flag, prm.timeout_ns);
-      if (ok) ok = mbar_wait(&ctrl->k_full[0], 0, abort_flag, prm.timeout_ns);
+      bool ok = mbar_wait_sleep(&ctrl->q_full, 0, abort_flag, prm.timeout_ns);
+      if (ok) ok = mbar_wait_sleep(&ctrl->k_full[0], 0, abort_flag, prm.timeout_ns);
       if (ok) {
         tc_fence_after();
         issue_qk(0, 0);
@@ -234,22 +238,22 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         const int vb = j & 1;
-        ok = mbar_wait(&ctrl->vh_full[vb], (j >> 1) & 1, abort_flag, prm.timeout_ns);
+        ok = mbar_wait_sleep(&ctrl->vh_full[vb], (j >> 1) & 1, abort_flag, prm.timeout_ns);
         if (!ok) break;
         const bool has_next = j + 1 < n_kv;
         const int ks = (j + 1) % kKStages;
-        ok = mbar_wait(&ctrl->p_full[0], j & 1, abort_flag, prm.timeout_ns);
+        ok = mbar_wait_sleep(&ctrl->p_full[0], j & 1, abort_flag, prm.timeout_ns);
         if (!ok) break;
         tc_fence_after();
         issue_pv(0, vb, j > 0);
         if (has_next) {
-          ok = mbar_wait(&ctrl->k_full[ks], ((j + 1) / kKStages) & 1, abort_flag, prm.timeout_ns);
+          ok = mbar_wait_sleep(&ctrl->k_full[ks], ((j + 1) / kKStages) & 1, abort_flag, prm.timeout_ns);
           if (!ok) break;
           tc_fence_after();
           issue_qk(0, ks);
           mma_commit(&ctrl->s_full[0]);
         }
-        ok = mbar_wait(&ctrl->p_full[1], j & 1, abort_flag, prm.timeout_ns);
+        ok = mbar_wait_sleep(&ctrl->p_full[1], j & 1, abort_flag, prm.timeout_ns);
         if (!ok) break;
         tc_fence_after();
         issue_pv(1, vb, j > 0);
@@ -282,20 +286,24 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (m > 0.f) {
         frexpf(m, &e);  // m = f * 2^e, f in [0.5, 1)  ->  2^e > m
       }
-      ctrl->v_log2_norm = static_cast<float>(e);
-      ctrl->v_norm = ldexpf(1.0f, e);
+      ctrl->v_norm = ldexpf(1.0f, e - 7);  // > max sv / 128
     }
     named_bar_sync(1, kCvtThreads);
+    const float inv_norm = 1.0f / ctrl->v_norm;  // a power of two: exact
     mbar_arrive(&ctrl->norm_ready);
 
     const uint8_t* vsrc_base = smem + kSmemV;
     for (int j = 0; j < n_kv; ++j) {
       const int vs = j % kVStages, vb = j & 1;
-      bool ok = mbar_wait(&ctrl->v_full[vs], (j / kVStages) & 1, abort_flag, prm.timeout_ns);
-      ok = ok && mbar_wait(&ctrl->vh_empty[vb], ((j >> 1) & 1) ^ 1, abort_flag, prm.timeout_ns);
+      bool ok = mbar_wait_sleep(&ctrl->v_full[vs], (j / kVStages) & 1, abort_flag, prm.timeout_ns);
+      ok = ok && mbar_wait_sleep(&ctrl->vh_empty[vb], ((j >> 1) & 1) ^ 1, abort_flag, prm.timeout_ns);
       if (!ok) break;
       const uint8_t* src = vsrc_base + vs * kTile8;
       uint8_t* dst = smem + kSmemVh + vb * kTile16;
+      // Block factors sv / 2^e of this tile's two 64-key blocks (a partial
+      // last tile reads the last block's scale for its zero-filled rows).
+      const __half2 f_lo = __float2half2_rn(__ldg(prm.v_scale + scale_row + 2 * j) * inv_norm);
+      const __half2 f_hi = __float2half2_rn(__ldg(prm.v_scale + scale_row + min(2 * j + 1, prm.nblk - 1)) * inv_norm);
 #pragma unroll 4
       for (int i = 0; i < (kBN * 8) / kCvtThreads; ++i) {
         // 16-byte source chunk (row r, channel chunk c16).  Consecutive lanes
@@ -305,7 +313,7 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int r = idx & (kBN - 1), c16 = idx >> 7;
         const uint4 raw = *reinterpret_cast<const uint4*>(src + r * 128 + ((c16 ^ (r & 7)) << 4));
         uint4 lo, hi;
-        widen16(raw, lo, hi);
+        widen16_scaled(raw, r < 64 ? f_lo : f_hi, lo, hi);
         const int box = c16 >> 2;             // channels 16*c16.. -> 64-channel box
         const int c8 = (c16 & 3) * 2;         // first 8-channel chunk inside the box
         uint8_t* row = dst + box * kBox16 + r * 128;
@@ -328,7 +336,6 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float sq = row < N ? __ldg(prm.q_scale + scale_row + row / 64) * prm.scale_log2 : 0.f;
 
     bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->norm_ready, 0, abort_flag, prm.timeout_ns));
-    const float lg_norm = ctrl->v_log2_norm;
     const float v_norm = ctrl->v_norm;
 
     float m = -INFINITY;
@@ -338,11 +345,6 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int kb0 = 2 * j, kb1 = min(2 * j + 1, prm.nblk - 1);
       const float c0 = sq * __ldg(prm.k_scale + scale_row + kb0);
       const float c1 = sq * __ldg(prm.k_scale + scale_row + kb1);
-      const float sv0 = __ldg(prm.v_scale + scale_row + kb0);
-      const float sv1 = __ldg(prm.v_scale + scale_row + kb1);
-      // Per-half constants that do not depend on S, formed before the wait.
-      const float lb0 = __log2f(sv0) - lg_norm, lb1 = __log2f(sv1) - lg_norm;
-      const float vi0 = v_norm / sv0, vi1 = v_norm / sv1;
       if (!__all_sync(0xffffffffu,
                       mbar_wait(&ctrl->s_full[t], static_cast<uint32_t>(j) & 1u, abort_flag, prm.timeout_ns))) {
         ok = false;
@@ -376,31 +378,27 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         l *= corr;
         m = mnew;
       }
-      // Exponent biases fold the V block scales: P' = P * sv / 2^e.
-      const float bias0 = lb0 - m;
-      const float bias1 = lb1 - m;
-      float l0, l1;
-      exp_pack_tile<true, kPolyEvery, false>(sv, c0, bias0, c1, bias1, nvalid >= kBN, l0, l1);
-      // Undo the V-scale fold for the row sum: sum P = sum P' * 2^e / sv.
-      l += l0 * vi0 + (nvalid > 64 ? l1 * vi1 : 0.f);
+      exp_pack_only<true>(sv, c0, -m, c1, -m);
       tmem_st32(s_addr, sv[0]);
       tmem_st32(s_addr + 32, sv[2]);
       // O correction after P is out of registers (keeps register pressure
       // down); it only has to land before this tile's P.V is issued.
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(o_addr + c * 32, ov);
-          tmem_ld_wait(ov);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t ov[16];
+          tmem_ld16(o_addr + c * 16, ov);
+          tmem_ld_wait16(ov);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-          tmem_st32(o_addr + c * 32, ov);
+          for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+          tmem_st16(o_addr + c * 16, ov);
         }
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctrl->p_full[t]);
+      // Row sum of the FP16 P the MMA multiplies V by, after the hand-off.
+      l += sum_packed<true>(sv[0]) + sum_packed<true>(sv[2]);
     }
 
     if (ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->o_full, 0, abort_flag, prm.timeout_ns))) {

@@ -97,3 +97,44 @@ def test_fp8_pipeline_t2i_2048_sampled(cuda_ok):
     qkv8, unq = _oracle_quant(w, q, k, v)
     codes, scales = zip(*qkv8)
     _check(w, o, lse, codes, scales, rows=I.sampled_rows(w, 256), unquant=unq)
+
+
+def _prologue_like_codes(w, seed, v_scale_fn):
+    """Q, K, V codes as the prologue would write them for N(0,1) rows (random
+    finite E4M3 codes would do too) with V block scales chosen by
+    ``v_scale_fn(nblk, rng)``; Q and K keep ordinary scales."""
+    rng = np.random.default_rng(seed)
+    nblk = -(-w.N // 64)
+    codes = [I.random_e4m3_codes((w.B, w.N, w.H, w.d), seed=seed + i) for i in range(3)]
+    scales = [np.exp(rng.uniform(-5.5, -4.5, (w.B, w.H, nblk))).astype(np.float32) for _ in range(2)]
+    scales.append(v_scale_fn(nblk, rng).astype(np.float32))
+    return codes, scales
+
+
+def test_fp8_all_zero_v_block(cuda_ok):
+    """One 64-token V block is all zero (the prologue then stores scale 1
+    and zero codes) while every other V block has a scale near 1e-2: the
+    zero block must not cost the other blocks precision."""
+    w = I.custom("zero_v", B=1, H=2, n_txt=64, img_h=16, img_w=20)
+
+    def v_scales(nblk, rng):
+        s = np.full((w.B, w.H, nblk), 0.01, dtype=np.float64) * np.exp(rng.uniform(-0.3, 0.3, (w.B, w.H, nblk)))
+        s[:, :, 2] = 1.0
+        return s
+
+    codes, scales = _prologue_like_codes(w, 41, v_scales)
+    codes[2][:, 128:192] = 0  # block 2 of every (b, h): zero codes, scale 1
+    o, lse = _gpu_fwd_fp8(w, codes, scales)
+    _check(w, o, lse, codes, scales)
+
+
+def test_fp8_v_scales_spanning_three_decades(cuda_ok):
+    """V block scales from 1e-4 to 1e-1 within each (b, h)."""
+    w = I.custom("spread_v", B=2, H=2, n_txt=30, img_h=10, img_w=30)
+
+    def v_scales(nblk, rng):
+        return 10.0 ** rng.uniform(-4.0, -1.0, (w.B, w.H, nblk))
+
+    codes, scales = _prologue_like_codes(w, 43, v_scales)
+    o, lse = _gpu_fwd_fp8(w, codes, scales)
+    _check(w, o, lse, codes, scales)
