@@ -1,8 +1,8 @@
 """Ulysses path on one GPU: a one-rank NCCL group, the all-to-all exchanges
 and the jattn prologue + BF16 attention on the head shard.  With one rank the
 exchanges are layout round trips, so the result must equal the direct
-library call bit for bit (the direct call is checked against the oracle in
-test_gpu_attn_bf16.py)."""
+library call bit for bit, and it must match the float64 oracle within the
+BF16 tolerances."""
 
 import os
 
@@ -13,6 +13,7 @@ import torch.distributed as dist
 from diffusion_transformer_joint_dit_b200 import binding as J
 from diffusion_transformer_joint_dit_b200 import inputs as I
 from diffusion_transformer_joint_dit_b200 import ulysses as U
+from tests.gpu_common import check_attention, oracle_prologue_bf16, to_np
 
 
 @pytest.fixture(scope="module")
@@ -38,3 +39,8 @@ def test_ulysses_one_rank_equals_direct(nccl_group, name):
     torch.cuda.synchronize()
     assert J.jattn_device_status() == J.JATTN_OK
     assert torch.equal(got, want)
+    # And against the float64 oracle chain (prologue, bf16 rounding,
+    # attention) on every row of tiny, 256 sampled rows of t2i_1024.
+    rows = None if w.N <= 512 else I.sampled_rows(w, 256)
+    _, _, qb, kb = oracle_prologue_bf16(w, q.cpu(), k.cpu())
+    check_attention(w, got, None, qb, kb, to_np(v), rows=rows)
