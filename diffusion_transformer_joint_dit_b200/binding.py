@@ -33,7 +33,7 @@ JATTN_SPARSE_KBLOCK = 128
 EXPORTED = ("jattn_prologue", "jattn_fwd_bf16", "jattn_fwd_fp8", "jattn_rope_table", "jattn_qkv_fused",
             "jattn_fp8_repair_select", "jattn_fp8_repair_apply", "jattn_sparse_select", "jattn_fwd_bf16_sparse",
             "jattn_status_string", "jattn_device_status", "jattn_selftest_wait_timeout",
-            "jattn_selftest_exp2_poly", "jattn_last_cuda_error", "jattn_sparse_select_noalloc")
+            "jattn_last_cuda_error", "jattn_sparse_select_noalloc")
 
 
 class JattnError(RuntimeError):
@@ -115,8 +115,6 @@ def load_library():
     lib.jattn_device_status.restype = _I
     lib.jattn_selftest_wait_timeout.argtypes = [ctypes.c_longlong, _P]
     lib.jattn_selftest_wait_timeout.restype = _I
-    lib.jattn_selftest_exp2_poly.argtypes = [_P, _P, _I, _P]
-    lib.jattn_selftest_exp2_poly.restype = _I
     lib.jattn_last_cuda_error.argtypes = []
     lib.jattn_last_cuda_error.restype = ctypes.c_char_p
     _lib = lib
@@ -309,11 +307,4 @@ def jattn_selftest_wait_timeout(timeout_ns: int, stream=None, *, check: bool = T
     st = load_library().jattn_selftest_wait_timeout(int(timeout_ns), _stream(stream))
     if check:
         _check("jattn_selftest_wait_timeout", st)
-    return st
-
-
-def jattn_selftest_exp2_poly(x, y, n: int, stream=None, *, check: bool = True) -> int:
-    st = load_library().jattn_selftest_exp2_poly(_ptr(x), _ptr(y), int(n), _stream(stream))
-    if check:
-        _check("jattn_selftest_exp2_poly", st)
     return st

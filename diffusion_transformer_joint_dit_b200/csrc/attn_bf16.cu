@@ -33,8 +33,10 @@
 // 128) are masked to -inf; tail query rows read zero-filled Q and are not
 // stored.
 //
-// The row sum is formed after P is handed to the MMA issuer, off the path
-// to the next P.V.  The producer and MMA threads wait with suspending
+// The row sum is the fp32 sum of the unrounded P plus the bf16 rounding of
+// each tile's largest P, so that a dominant key carries the same weight in
+// O = sum bf16(P) V and in l; its last step follows the hand-off of P to
+// the MMA issuer.  The producer and MMA threads wait with suspending
 // mbarrier waits, so that they take no issue slots from the softmax warps
 // of their SM sub-partitions while they wait.
 //
@@ -322,9 +324,15 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         l *= corr;
         m = mnew;
       }
+      // Row sum: the fp32 sum of the unrounded P, plus the bf16 rounding of
+      // the tile's largest P (formed bit for bit as the packing loop forms
+      // it), so that a dominant key has the same weight in the numerator
+      // O = sum bf16(P) V and in l.
+      const float pm = ex2_approx(fmaf(fmaxf(mx_lo, mx_hi), sl2, -m));
+      const float fix = __bfloat162float(__float2bfloat16_rn(pm)) - pm;
       // P = exp2(s * scale * log2e - m), packed two bf16 per 32-bit word in
       // place: keys [0,64) land in sv[0], keys [64,128) in sv[2].
-      exp_pack_only<false>(sv, sl2, -m, sl2, -m);
+      const float lt = exp_pack_sum<false>(sv, sl2, -m, sl2, -m) + fix;
       tmem_st32(s_addr, sv[0]);
       tmem_st32(s_addr + 32, sv[2]);
       // O correction after P is out of registers (keeps register pressure
@@ -343,8 +351,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctrl->p_full[t]);
-      // Row sum of the rounded P, after the hand-off.
-      l += sum_packed<false>(sv[0]) + sum_packed<false>(sv[2]);
+      l += lt;
     }
 
     if (ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->o_full, 0, abort_flag, prm.timeout_ns))) {

@@ -10,7 +10,8 @@
 //   P     = exp2(x - m), written to TMEM as FP16;
 //   V16   = code * (sv(block) / 2^e), widened and scaled to FP16 in shared
 //           memory by the converter warps;
-//   O    += P . V16;  l = sum P (the FP16 values the MMA uses);
+//   O    += P . V16;  l = sum P (fp32; the largest P of each tile counted
+//           as the FP16 value the MMA uses);
 //   O     = O * 2^e / l.
 //
 // The per-(b, h) power of two 2^e >= max_block sv / 128 keeps |V16| <=
@@ -378,7 +379,12 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         l *= corr;
         m = mnew;
       }
-      exp_pack_only<true>(sv, c0, -m, c1, -m);
+      // Row sum: fp32 sum of the unrounded P plus the fp16 rounding of the
+      // tile's largest P (formed as the packing loop forms it), so that a
+      // dominant key has the same weight in O = sum fp16(P) V16 and in l.
+      const float pm = ex2_approx(fmaxf(fmaf(mx_lo, c0, -m), fmaf(mx_hi, c1, -m)));
+      const float fix = __half2float(__float2half_rn(pm)) - pm;
+      const float lt = exp_pack_sum<true>(sv, c0, -m, c1, -m) + fix;
       tmem_st32(s_addr, sv[0]);
       tmem_st32(s_addr + 32, sv[2]);
       // O correction after P is out of registers (keeps register pressure
@@ -397,8 +403,7 @@ attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ctrl->p_full[t]);
-      // Row sum of the FP16 P the MMA multiplies V by, after the hand-off.
-      l += sum_packed<true>(sv[0]) + sum_packed<true>(sv[2]);
+      l += lt;
     }
 
     if (ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->o_full, 0, abort_flag, prm.timeout_ns))) {

@@ -55,17 +55,6 @@ __global__ void wait_selftest_kernel(uint64_t timeout_ns) {
   __syncthreads();
 }
 
-// Polynomial-exp2 self test: pairs of inputs through the softmax's helper.
-__global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float a = x[i];
-  const float b = i + 1 < n ? x[i + 1] : 0.f;
-  const uint64_t r = exp2_poly2(f2_pack(a, b));
-  y[i] = f2_lo(r);
-  if (i + 1 < n) y[i + 1] = f2_hi(r);
-}
-
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
 
 thread_local cudaError_t t_last_cuda_error = cudaSuccess;
@@ -513,14 +502,6 @@ int jattn_device_status(void* cuda_stream) {
 int jattn_selftest_wait_timeout(long long timeout_ns, void* cuda_stream) {
   if (timeout_ns < 1 || timeout_ns > 1000000000ll) return JATTN_ERR_INVALID_ARG;
   return map_err(launch_wait_selftest(static_cast<uint64_t>(timeout_ns), static_cast<cudaStream_t>(cuda_stream)));
-}
-
-int jattn_selftest_exp2_poly(const float* x, float* y, int n, void* cuda_stream) {
-  if (x == nullptr || y == nullptr || n < 1) return JATTN_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 7u) return JATTN_ERR_MISALIGNED;
-  const int pairs = (n + 1) / 2;
-  exp2_poly_selftest_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(cuda_stream)>>>(x, y, n);
-  return map_err(cudaGetLastError());
 }
 
 }  // extern "C"

@@ -193,18 +193,22 @@ __global__ void __launch_bounds__(kBf16Warps * 32) prologue_bf16_kernel(const __
 // table of a block (cos, sin of its 64 tokens x 64 channel pairs, 32 KB of
 // shared memory) is built once and reused for every head pair of the block.
 // An item's Q, K and V rows (64 tokens x 2 heads x 256 B = 32 KB each) come
-// in by TMA into one of two shared-memory buffers; the next item's rows
-// land while this one is processed, so HBM stays busy.
+// in by TMA into one of two shared-memory buffers.  Every warp copies its
+// rows of the item into registers first and then arrives on the buffer's
+// `empty` barrier, so thread 0 can refill the buffer with the next-but-one
+// item while the arithmetic of this one runs.
 // Warp w handles head w / 8 of the pair and tokens [8 (w mod 8), +8), a
-// half-warp per row: each lane keeps 4 rows of 8 channels in registers
-// from normalisation to quantisation (16 warps per SM hide the latency of
-// the shuffles and conversions).  The block absmax needs every processed
-// value of the block: each warp reduces its 8 tokens, the eight warps of a
-// head meet through shared memory and a 256-thread named barrier, then all
-// quantise from registers.
+// half-warp per row: each lane keeps 4 rows of 8 channels of Q, K and V in
+// registers from normalisation to quantisation.  The block absmax needs
+// every processed value of the block: each warp reduces its 8 tokens of Q,
+// K and V (one redux.sync each), and the eight warps of a head exchange the
+// three partial maxima through shared memory at one named barrier per item.
+// The exchange slots alternate between items, so no second barrier is
+// needed before they are rewritten.
 constexpr int kF8Pair = 2;                                       // heads per item
 constexpr int kF8WarpsPerHead = 8;
-constexpr int kF8Threads = kF8Pair * kF8WarpsPerHead * 32;       // 512
+constexpr int kF8Warps = kF8Pair * kF8WarpsPerHead;              // 16
+constexpr int kF8Threads = kF8Warps * 32;                        // 512
 constexpr int kF8Rows = kQuantBlock / (2 * kF8WarpsPerHead);     // 4 rows per lane
 constexpr int kF8TileBytes = kQuantBlock * kF8Pair * kHeadDim * 2;  // 32 KB
 constexpr int kF8SmemRot = 0;                                    // float2 [64][64]
@@ -219,6 +223,14 @@ __device__ __forceinline__ uint32_t absmax8_u16x2(const uint4& u, uint32_t m) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) asm("max.u16x2 %0, %0, %1;" : "+r"(m) : "r"(w[i] & 0x7FFF7FFFu));
   return m;
+}
+
+// Warp-wide maximum of a non-negative float: non-negative IEEE floats order
+// like their bit patterns as unsigned integers.
+__device__ __forceinline__ float warp_max_nonneg(float x) {
+  uint32_t u;
+  asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(u) : "r"(__float_as_uint(x)));
+  return __uint_as_float(u);
 }
 
 __device__ __forceinline__ uint2 quant8(const uint4& u, float inv) {
@@ -249,8 +261,10 @@ prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constan
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float2 (*s_rot)[64] = reinterpret_cast<float2 (*)[64]>(smem + kF8SmemRot);  // [token][axis * 32 + pair]
-  __shared__ uint64_t s_full[2][3];            // [buffer][Q, K, V] rows landed
-  __shared__ float s_amax[kF8Pair][kF8WarpsPerHead];  // [head of the pair][warp of the head]
+  __shared__ uint64_t s_full[2];   // the buffer's Q, K, V rows have landed
+  __shared__ uint64_t s_empty[2];  // every warp has copied the buffer's rows into registers
+  // Partial block maxima: [item parity][head of the pair][Q, K, V][warp of the head].
+  __shared__ __align__(16) float s_amax[2][kF8Pair][3][kF8WarpsPerHead];
   __shared__ int s_abort;
 
   const int warp = threadIdx.x >> 5;
@@ -280,17 +294,21 @@ prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constan
   auto issue = [&](int item, int buf) {
     int blk, b, hp;
     coords(item, blk, b, hp);
+    mbar_arrive_expect_tx(&s_full[buf], 3 * kF8TileBytes);
 #pragma unroll
-    for (int x = 0; x < 3; ++x) {
-      mbar_arrive_expect_tx(&s_full[buf][x], kF8TileBytes);
-      tma_load_4d(tile(buf, x), maps[x], &s_full[buf][x], 0, hp * kF8Pair, blk * kQuantBlock, b);
-    }
+    for (int x = 0; x < 3; ++x) tma_load_4d(tile(buf, x), maps[x], &s_full[buf], 0, hp * kF8Pair, blk * kQuantBlock, b);
   };
+
+  float wq[8], wk[8];
+  load_weights(a.q_w, l16, wq);
+  load_weights(a.k_w, l16, wk);
 
   int issued_end = begin;  // thread 0: one past the last item whose copies were issued
   if (threadIdx.x == 0) {
-    for (int u = 0; u < 2; ++u)
-      for (int x = 0; x < 3; ++x) mbar_init(&s_full[u][x], 1);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&s_full[u], 1);
+      mbar_init(&s_empty[u], kF8Warps);
+    }
     s_abort = 0;
     fence_barrier_init();
     if (begin < end) {
@@ -307,16 +325,22 @@ prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constan
   for (int item = begin; item < end; ++item) {
     const int i = item - begin;
     const int buf = i & 1;
-    // Buffer buf ^ 1 was released by the barrier that ended the previous item.
+    // Refill the other buffer with the next item once every warp has copied
+    // item i - 1's rows out of it (its i-th use is phase i >> 1).
     if (threadIdx.x == 0 && item + 1 < end && !s_abort) {
-      issue(item + 1, buf ^ 1);
-      issued_end = item + 2;
+      const bool free = i == 0 || mbar_wait(&s_empty[buf ^ 1], static_cast<uint32_t>((i - 1) >> 1) & 1u, &s_abort,
+                                            a.timeout_ns);
+      if (free) {
+        issue(item + 1, buf ^ 1);
+        issued_end = item + 2;
+      }
     }
     int blk, b, hp;
     coords(item, blk, b, hp);
     const int t0 = blk * kQuantBlock;
     const int h = hp * kF8Pair + hl;
     if (blk != cur_blk) {  // same for the whole CTA
+      __syncthreads();     // every warp is done with the previous block's table
       for (int e = threadIdx.x; e < kQuantBlock * 64; e += kF8Threads) {
         const int tok = e >> 6, pr = e & 63;
         int row = 0, col = 0;
@@ -331,65 +355,82 @@ prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constan
       cur_blk = blk;
     }
 
-#pragma unroll 1
+    const bool ok = mbar_wait(&s_full[buf], static_cast<uint32_t>(i >> 1) & 1u, &s_abort, a.timeout_ns);
+    uint4 rows[3][kF8Rows];  // [Q, K, V][row]
+#pragma unroll
     for (int x = 0; x < 3; ++x) {
-      const bool ok = mbar_wait(&s_full[buf][x], static_cast<uint32_t>(i >> 1) & 1u, &s_abort, a.timeout_ns);
       const uint4* src = reinterpret_cast<const uint4*>(tile(buf, x));
-      uint4 rows[kF8Rows];
 #pragma unroll
       for (int r = 0; r < kF8Rows; ++r)
-        rows[r] = ok ? src[((tok0 + 2 * r) * kF8Pair + hl) * 16 + l16] : make_uint4(0, 0, 0, 0);
-      float amax = 0.f;
-      if (x < 2) {
-        float w[8];
-        load_weights(x == 0 ? a.q_w : a.k_w, l16, w);
+        rows[x][r] = ok ? src[((tok0 + 2 * r) * kF8Pair + hl) * 16 + l16] : make_uint4(0, 0, 0, 0);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s_empty[buf]);
+
+    // Q and K: RMSNorm, weight, rotation (one table read per row serves
+    // both), and the block maxima of the bf16 results over valid tokens.
+    float amax[3] = {0.f, 0.f, 0.f};
 #pragma unroll
-        for (int r = 0; r < kF8Rows; ++r) {
-          const int tok = tok0 + 2 * r;
-          const float4 r0 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0]);
-          const float4 r1 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0 + 2]);
-          const float c[4] = {r0.x, r0.z, r1.x, r1.z};
-          const float sn[4] = {r0.y, r0.w, r1.y, r1.w};
-          float am = 0.f;
-          rows[r] = norm_rope_row_amax(rows[r], w, c, sn, a.eps, am);
-          amax = t0 + tok < a.N ? fmaxf(amax, am) : amax;
-        }
-        amax = __bfloat162float(__float2bfloat16_rn(amax));
-      } else {
-        uint32_t m2 = 0;
-#pragma unroll
-        for (int r = 0; r < kF8Rows; ++r) m2 = absmax8_u16x2(rows[r], m2);
-        amax = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+    for (int r = 0; r < kF8Rows; ++r) {
+      const int tok = tok0 + 2 * r;
+      const float4 r0 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0]);
+      const float4 r1 = *reinterpret_cast<const float4*>(&s_rot[tok][axis * 32 + pair0 + 2]);
+      const float c[4] = {r0.x, r0.z, r1.x, r1.z};
+      const float sn[4] = {r0.y, r0.w, r1.y, r1.w};
+      float aq = 0.f, ak = 0.f;
+      rows[0][r] = norm_rope_row_amax(rows[0][r], wq, c, sn, a.eps, aq);
+      rows[1][r] = norm_rope_row_amax(rows[1][r], wk, c, sn, a.eps, ak);
+      if (t0 + tok < a.N) {
+        amax[0] = fmaxf(amax[0], aq);
+        amax[1] = fmaxf(amax[1], ak);
       }
+    }
+    amax[0] = __bfloat162float(__float2bfloat16_rn(amax[0]));
+    amax[1] = __bfloat162float(__float2bfloat16_rn(amax[1]));
+    {
+      uint32_t m2 = 0;  // V: max |v| of the bf16 inputs (rows past N are zero-filled)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      if (lane == 0) s_amax[hl][tq] = amax;
-      named_bar_sync(bar_id, kF8WarpsPerHead * 32);
+      for (int r = 0; r < kF8Rows; ++r) m2 = absmax8_u16x2(rows[2][r], m2);
+      amax[2] = fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+    }
+    float(*slot)[kF8WarpsPerHead] = s_amax[i & 1][hl];
 #pragma unroll
-      for (int k = 0; k < kF8WarpsPerHead; ++k) amax = fmaxf(amax, s_amax[hl][k]);
-      named_bar_sync(bar_id, kF8WarpsPerHead * 32);  // all read before s_amax is rewritten
-      if (ok && h < a.H) {
-        const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 0.f;
+    for (int x = 0; x < 3; ++x) {
+      const float m = warp_max_nonneg(amax[x]);
+      if (lane == 0) slot[x][tq] = m;
+    }
+    named_bar_sync(bar_id, kF8WarpsPerHead * 32);
+#pragma unroll
+    for (int x = 0; x < 3; ++x) {
+      const float4 lo = *reinterpret_cast<const float4*>(&slot[x][0]);
+      const float4 hi = *reinterpret_cast<const float4*>(&slot[x][4]);
+      amax[x] = fmaxf(fmax3(lo.x, lo.y, fmax3(lo.z, lo.w, hi.x)), fmax3(hi.y, hi.z, hi.w));
+    }
+
+    if (ok && h < a.H) {
+#pragma unroll
+      for (int x = 0; x < 3; ++x) {
+        const float inv = amax[x] > 0.f ? __fdiv_rn(448.0f, amax[x]) : 0.f;
         if (tq == 0 && lane == 0) {
           float* sc = x == 0 ? a.q_scale : (x == 1 ? a.k_scale : a.v_scale);
-          sc[(static_cast<size_t>(b) * a.H + h) * nblk + blk] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+          sc[(static_cast<size_t>(b) * a.H + h) * nblk + blk] = amax[x] > 0.f ? __fdiv_rn(amax[x], 448.0f) : 1.0f;
         }
         uint2* out = reinterpret_cast<uint2*>(x == 0 ? a.q_out : (x == 1 ? a.k_out : a.v_out));
 #pragma unroll
         for (int r = 0; r < kF8Rows; ++r) {
           const int t = t0 + tok0 + 2 * r;
-          if (t < a.N) __stcs(out + ((static_cast<size_t>(b) * a.N + t) * a.H + h) * 16 + l16, quant8(rows[r], inv));
+          if (t < a.N) __stcs(out + ((static_cast<size_t>(b) * a.N + t) * a.H + h) * 16 + l16, quant8(rows[x][r], inv));
         }
       }
     }
-    __syncthreads();  // buffer buf and the table are free again
   }
-  // Drain: the last two issued items' copies have landed before the CTA exits.
+  // Drain: the copies of the last two issued items have landed before the
+  // CTA exits (all of them, unless a wait timed out).
   if (threadIdx.x == 0) {
     int never = 0;
     for (int item = (issued_end - 2 > begin ? issued_end - 2 : begin); item < issued_end; ++item) {
       const int i = item - begin;
-      for (int x = 0; x < 3; ++x) mbar_wait(&s_full[i & 1][x], static_cast<uint32_t>(i >> 1) & 1u, &never, a.timeout_ns);
+      mbar_wait(&s_full[i & 1], static_cast<uint32_t>(i >> 1) & 1u, &never, a.timeout_ns);
     }
   }
 }

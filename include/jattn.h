@@ -422,17 +422,6 @@ JATTN_API int jattn_device_status(void* cuda_stream);
  */
 JATTN_API int jattn_selftest_wait_timeout(long long timeout_ns, void* cuda_stream);
 
-/*
- * jattn_selftest_exp2_poly — evaluate, for n floats x (device pointers), the
- * range-reduced polynomial exp2 the attention softmax can use for a share of
- * its exponentials (built in, switched off: all-MUFU measured faster),
- * writing y[i] ~ 2^x[i].  Lets tests check its error bound
- * (relative 7.5e-5 from the degree-3 minimax fit, for x in [-125, 8];
- * smaller x is clamped to -125).
- * n >= 1; x and y 8-byte aligned; asynchronous on cuda_stream.
- */
-JATTN_API int jattn_selftest_exp2_poly(const float* x, float* y, int n, void* cuda_stream);
-
 #ifdef __cplusplus
 }
 #endif
