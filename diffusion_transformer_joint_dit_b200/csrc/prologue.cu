@@ -195,8 +195,9 @@ __global__ void __launch_bounds__(kBf16Warps * 32) prologue_bf16_kernel(const __
 // An item's Q, K and V rows (64 tokens x 2 heads x 256 B = 32 KB each) come
 // in by TMA into one of two shared-memory buffers.  Every warp copies its
 // rows of the item into registers first and then arrives on the buffer's
-// `empty` barrier, so thread 0 can refill the buffer with the next-but-one
-// item while the arithmetic of this one runs.
+// `empty` barrier; thread 0 refills the buffer with the next-but-one item
+// as soon as all have, so two items' copies are in flight while the
+// arithmetic of this one runs.
 // Warp w handles head w / 8 of the pair and tokens [8 (w mod 8), +8), a
 // half-warp per row: each lane keeps 4 rows of 8 channels of Q, K and V in
 // registers from normalisation to quantisation.  The block absmax needs
@@ -315,6 +316,10 @@ prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constan
       for (int x = 0; x < 3; ++x) prefetch_tensormap(maps[x]);
       issue(begin, 0);
       issued_end = begin + 1;
+      if (begin + 1 < end) {
+        issue(begin + 1, 1);
+        issued_end = begin + 2;
+      }
     }
   }
   __syncthreads();
@@ -325,16 +330,6 @@ prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constan
   for (int item = begin; item < end; ++item) {
     const int i = item - begin;
     const int buf = i & 1;
-    // Refill the other buffer with the next item once every warp has copied
-    // item i - 1's rows out of it (its i-th use is phase i >> 1).
-    if (threadIdx.x == 0 && item + 1 < end && !s_abort) {
-      const bool free = i == 0 || mbar_wait(&s_empty[buf ^ 1], static_cast<uint32_t>((i - 1) >> 1) & 1u, &s_abort,
-                                            a.timeout_ns);
-      if (free) {
-        issue(item + 1, buf ^ 1);
-        issued_end = item + 2;
-      }
-    }
     int blk, b, hp;
     coords(item, blk, b, hp);
     const int t0 = blk * kQuantBlock;
@@ -366,6 +361,13 @@ prologue_fp8_kernel(const __grid_constant__ PrologueArgs a, const __grid_constan
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&s_empty[buf]);
+    // Refill this buffer with item i + 2 once every warp has copied item i's
+    // rows out of it (the buffer's (i >> 1)-th use).
+    if (threadIdx.x == 0 && item + 2 < end && !s_abort &&
+        mbar_wait(&s_empty[buf], static_cast<uint32_t>(i >> 1) & 1u, &s_abort, a.timeout_ns)) {
+      issue(item + 2, buf);
+      issued_end = item + 3;
+    }
 
     // Q and K: RMSNorm, weight, rotation (one table read per row serves
     // both), and the block maxima of the bf16 results over valid tokens.
