@@ -545,6 +545,21 @@ def time_qkv_fused(J, dev, stream, rank: int, peaks, peaks_src, steps: int = 10)
     }
 
 
+def sm_count(dev) -> int:
+    return torch.cuda.get_device_properties(dev).multi_processor_count
+
+
+def attn_bf16_launches(B: int, H: int, N: int, sms: int) -> int:
+    """Kernel launches of one jattn_fwd_bf16 call: one over the whole waves
+    of 256-row work items (one CTA per SM), plus one for a last partial wave
+    that fills at most half of the SMs, which runs split over KV halves."""
+    n_qb, n_kv = -(-N // 256), -(-N // 128)
+    items = n_qb * H * B
+    rem = items % sms
+    tail = rem if n_kv >= 2 and 2 * rem <= sms else 0
+    return int(items - tail > 0) + int(tail > 0)
+
+
 def mufu_roofline(w: I.Workload, att_ms: float, clocks, dev):
     """Secondary roofline of the attention kernel: one exp2 per score
     (B H N^2 per launch) against the SFU rate, 16 ex2 per clock per SM (a
@@ -780,7 +795,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 3 * act_bytes,
                 "d2h_bytes_per_step": act_bytes, "steps": Ke,
                 "note": "copies of neighbouring steps overlap compute (H2D, compute, D2H streams)"},
-        "gpu_launches": 2 * K,
+        "gpu_launches": K * (1 + attn_bf16_launches(w.B, w.H, w.N, sm_count(dev))),
         "clocks": clocks,
     }
     if world > 1:
@@ -912,7 +927,7 @@ def run_cfg_ulysses(args, rank: int, world: int, local_rank: int):
                     "all_to_all_bytes_sent_per_rank_per_step":
                         4 * nb * (s1 - s0) * w.H * w.d * 2 * (layout.sp - 1) // layout.sp,
                     "l2": "inputs larger than L2"}),
-                "gpu_launches": 2 * K,
+                "gpu_launches": K * (1 + attn_bf16_launches(nb, hp, w.N, sm_count(dev))),
                 "clocks": clk,
             }
             print(json.dumps(line), flush=True)

@@ -40,6 +40,16 @@
 // mbarrier waits, so that they take no issue slots from the softmax warps
 // of their SM sub-partitions while they wait.
 //
+// Split tail (kSplit): a launch covers whole waves of work items (256
+// query rows of one (b, h)), one CTA per SM; the items of a last, partial
+// wave are run by a second launch in which a cluster of two CTAs shares an
+// item, each over half of the KV tiles.  At the end CTA 1 writes its
+// unnormalised O rows, m and l into CTA 0's (then idle) shared memory and
+// CTA 0 merges the two halves:
+//   m = max(m0, m1),  l = 2^(m0-m) l0 + 2^(m1-m) l1,
+//   O = (2^(m0-m) O0 + 2^(m1-m) O1) / l.
+// The partial wave then takes half as long.
+//
 // Block-sparse variant (kSparse): the tutorial's Sol-Attention runs a
 // generic block-sparse attention kernel.  A CTA's 256 query rows are one
 // query block; it visits only the KV tiles listed for that block (a count
@@ -76,6 +86,8 @@ struct Ctrl {
   uint64_t p_full[kTiles];
   uint64_t o_full;
   uint64_t mma_done;
+  uint64_t peer_free;     // split, CTA 1: CTA 0's shared memory may take the partial result
+  uint64_t partial_full;  // split, CTA 0: CTA 1's partial result has landed
   uint32_t tmem_base;
   int abort;
 };
@@ -84,6 +96,13 @@ constexpr int kSmemQ = 0;
 constexpr int kSmemRing = kTiles * kTileBytes;
 constexpr int kSmemCtrl = kSmemRing + kStages * kTileBytes;
 constexpr int kSmemBytes = kSmemCtrl + static_cast<int>(sizeof(Ctrl)) + 1024;  // + alignment slack
+// Split tail: CTA 1's partial result in CTA 0's Q + ring region, O as
+// [32 column quads][256 rows][4] fp32 (each thread's 16-byte stores land in
+// consecutive chunks), then m[256] and l[256].
+constexpr int kPartO = 0;
+constexpr int kPartM = kPartO + kTiles * kBM * kD * 4;  // 128 KB
+constexpr int kPartL = kPartM + kTiles * kBM * 4;
+static_assert(kPartL + kTiles * kBM * 4 <= kSmemCtrl, "partial result must fit below the barriers");
 
 struct Params {
   __nv_bfloat16* o;
@@ -91,6 +110,8 @@ struct Params {
   const int* kv_idx;  // block-sparse only: [B, H, n_qb, n_kv] tile lists
   const int* kv_cnt;  // block-sparse only: [B, H, n_qb] list lengths
   int H, N;
+  int n_qb;           // query blocks (256 rows) per (b, h)
+  int item0;          // first work item of this launch; item = (b * H + h) * n_qb + qb
   float scale_log2;
   uint64_t timeout_ns;
 };
@@ -101,7 +122,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint6
   return mbar_wait_sleep(bar, parity, &never, timeout_ns);
 }
 
-template <bool kSparse>
+template <bool kSparse, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Params prm) {
@@ -110,25 +131,38 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + kSmemCtrl);
   volatile int* abort_flag = &ctrl->abort;
 
+  // The split-tail launch that follows this one may start its CTAs as this
+  // grid's CTAs retire (programmatic dependent launch; no-op otherwise).
+  if constexpr (!kSplit) asm volatile("griddepcontrol.launch_dependents;");
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int m0 = blockIdx.x * (kBM * kTiles);
+  // Work item of this CTA (split: of its cluster; rank = CTA in the pair).
+  const int item = prm.item0 + static_cast<int>(kSplit ? blockIdx.x >> 1 : blockIdx.x);
+  const int rank = kSplit ? static_cast<int>(blockIdx.x & 1) : 0;
+  const int qb = item % prm.n_qb;
+  const int h = (item / prm.n_qb) % prm.H;
+  const int b = item / (prm.n_qb * prm.H);
+  const int m0 = qb * (kBM * kTiles);
   const int N = prm.N;
   const int n_kv = (N + kBN - 1) / kBN;
-  // KV tiles visited: all of them, or the query block's list.
+  // KV tiles visited: all of them, the query block's list, or (split) one
+  // half of them (the host splits only when n_kv >= 2).
   const int* list = nullptr;
   int n_iter = n_kv;
+  int kv0 = 0;
   if constexpr (kSparse) {
-    const size_t blk = (static_cast<size_t>(b) * prm.H + h) * gridDim.x + blockIdx.x;
-    list = prm.kv_idx + blk * n_kv;
-    n_iter = min(max(__ldg(prm.kv_cnt + blk), 0), n_kv);
+    list = prm.kv_idx + static_cast<size_t>(item) * n_kv;
+    n_iter = min(max(__ldg(prm.kv_cnt + item), 0), n_kv);
+  }
+  if constexpr (kSplit) {
+    const int half = (n_kv + 1) / 2;
+    kv0 = rank == 0 ? 0 : half;
+    n_iter = rank == 0 ? half : n_kv - half;
   }
   // Tile of the jj-th visit (clamped into range: memory-safe for any list).
   auto tile_of = [&](int jj) -> int {
     if constexpr (kSparse) return min(max(__ldg(list + jj), 0), n_kv - 1);
-    return jj;
+    return kv0 + jj;
   };
 
   if (threadIdx.x == 0) {
@@ -143,6 +177,8 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     mbar_init(&ctrl->o_full, 1);
     mbar_init(&ctrl->mma_done, 1);
+    mbar_init(&ctrl->peer_free, kTiles * kBM);     // every softmax thread of CTA 0
+    mbar_init(&ctrl->partial_full, kTiles * kBM);  // every softmax thread of CTA 1
     ctrl->abort = 0;
     fence_barrier_init();
   }
@@ -152,6 +188,7 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kSplit) cluster_sync();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
 
@@ -354,12 +391,57 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       l += lt;
     }
 
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->o_full, 0, abort_flag, prm.timeout_ns))) {
-      tc_fence_after();
-      const int row = m0 + t * kBM + r;
+    ok = ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->o_full, 0, abort_flag, prm.timeout_ns));
+    if (ok) tc_fence_after();
+    const int prow = t * kBM + r;  // row within the CTA's 256
+    float a_own = 1.f, a_peer = 0.f;  // split, CTA 0: weights of the two halves
+    bool store = ok;
+    if constexpr (kSplit) {
+      if (rank == 1) {
+        // Send the unnormalised O row, m and l to CTA 0 once its shared
+        // memory is idle (its MMAs and copies are complete).
+        store = false;
+        bool free = ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->peer_free, 0, abort_flag, prm.timeout_ns));
+        if (free) {
+          fence_acq_rel_cluster();
+          const uint32_t base = mapa_shared(smem_u32(smem), 0);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(o_addr + c * 32, ov);
+            tmem_ld_wait(ov);
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              st_cluster_v4(base + kPartO + (((c * 8 + q4) * (kTiles * kBM) + prow) << 4), ov[4 * q4], ov[4 * q4 + 1],
+                            ov[4 * q4 + 2], ov[4 * q4 + 3]);
+          }
+          st_cluster_f32(base + kPartM + prow * 4, m);
+          st_cluster_f32(base + kPartL + prow * 4, l);
+          mbar_arrive_cluster(mapa_shared(smem_u32(&ctrl->partial_full), 0));
+        }
+      } else {
+        // This CTA's Q and ring are idle: let CTA 1 write there, then merge.
+        mbar_arrive_cluster(mapa_shared(smem_u32(&ctrl->peer_free), 1));
+        store = ok && __all_sync(0xffffffffu, mbar_wait(&ctrl->partial_full, 0, abort_flag, prm.timeout_ns));
+        if (store) {
+          fence_acq_rel_cluster();
+          const float m1 = *reinterpret_cast<const float*>(smem + kPartM + prow * 4);
+          const float l1 = *reinterpret_cast<const float*>(smem + kPartL + prow * 4);
+          const float mm = fmaxf(m, m1);
+          a_own = ex2_approx(m - mm);
+          a_peer = ex2_approx(m1 - mm);
+          l = a_own * l + a_peer * l1;
+          m = mm;
+        }
+      }
+    }
+
+    if (store) {
+      const int row = m0 + prow;
       // l > 0 whenever a tile was visited (the row max contributes 1).
       const bool empty = kSparse && !(l > 0.f);
       const float inv_l = empty ? 0.f : 1.0f / l;
+      const float f_own = a_own * inv_l, f_peer = a_peer * inv_l;
       __nv_bfloat16* orow = prm.o + ((static_cast<size_t>(b) * N + row) * prm.H + h) * kD;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -372,15 +454,29 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int i = 0; i < 32; ++i) ov[i] = 0u;  // O's columns were never written
           }
         }
+        float o[32];
+        if constexpr (kSplit) {
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 pv = *reinterpret_cast<const float4*>(smem + kPartO + (((c * 8 + q4) * (kTiles * kBM) + prow) << 4));
+            o[4 * q4 + 0] = fmaf(__uint_as_float(ov[4 * q4 + 0]), f_own, pv.x * f_peer);
+            o[4 * q4 + 1] = fmaf(__uint_as_float(ov[4 * q4 + 1]), f_own, pv.y * f_peer);
+            o[4 * q4 + 2] = fmaf(__uint_as_float(ov[4 * q4 + 2]), f_own, pv.z * f_peer);
+            o[4 * q4 + 3] = fmaf(__uint_as_float(ov[4 * q4 + 3]), f_own, pv.w * f_peer);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(ov[i]) * inv_l;
+        }
         if (row < N) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(ov[8 * q4 + 0]) * inv_l, __uint_as_float(ov[8 * q4 + 1]) * inv_l);
-            u.y = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2]) * inv_l, __uint_as_float(ov[8 * q4 + 3]) * inv_l);
-            u.z = pack_bf16x2(__uint_as_float(ov[8 * q4 + 4]) * inv_l, __uint_as_float(ov[8 * q4 + 5]) * inv_l);
-            u.w = pack_bf16x2(__uint_as_float(ov[8 * q4 + 6]) * inv_l, __uint_as_float(ov[8 * q4 + 7]) * inv_l);
+            u.x = pack_bf16x2(o[8 * q4 + 0], o[8 * q4 + 1]);
+            u.y = pack_bf16x2(o[8 * q4 + 2], o[8 * q4 + 3]);
+            u.z = pack_bf16x2(o[8 * q4 + 4], o[8 * q4 + 5]);
+            u.w = pack_bf16x2(o[8 * q4 + 6], o[8 * q4 + 7]);
             dst[q4] = u;
           }
         }
@@ -394,10 +490,17 @@ attn_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   tc_fence_before();
   __syncthreads();
+  // Split: neither CTA of the pair leaves while the other may still touch
+  // its shared memory (every wait above is bounded, so both arrive).
+  if constexpr (kSplit) cluster_sync();
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  // Split tail: this grid may have started before the preceding one (the
+  // main launch) finished; it completes only after that one has, so that
+  // stream order holds for the work after the call.
+  if constexpr (kSplit) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace bf16attn
@@ -413,8 +516,10 @@ cudaError_t launch_bf16(const AttnProblem& p, const int* kv_idx, const int* kv_c
   if ((e = make_act_map(&tq, p.q, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
   if ((e = make_act_map(&tk, p.k, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
   if ((e = make_act_map(&tv, p.v, p.B, p.N, p.H, 2)) != cudaSuccess) return e;
-  if ((e = set_smem_attr(reinterpret_cast<const void*>(attn_bf16_kernel<kSparse>), kSmemBytes)) != cudaSuccess)
-    return e;
+  const int n_qb = (p.N + kBM * kTiles - 1) / (kBM * kTiles);
+  const int n_kv = (p.N + kBN - 1) / kBN;
+  const long long n_items = static_cast<long long>(n_qb) * p.H * p.B;
+  if (n_items > 0x3fffffff) return cudaErrorInvalidValue;
   Params prm;
   prm.o = static_cast<__nv_bfloat16*>(p.o);
   prm.lse = p.lse;
@@ -422,10 +527,51 @@ cudaError_t launch_bf16(const AttnProblem& p, const int* kv_idx, const int* kv_c
   prm.kv_cnt = kv_cnt;
   prm.H = p.H;
   prm.N = p.N;
+  prm.n_qb = n_qb;
+  prm.item0 = 0;
   prm.scale_log2 = static_cast<float>(static_cast<double>(p.softmax_scale) * 1.4426950408889634074);
   prm.timeout_ns = p.timeout_ns;
-  dim3 grid((p.N + kBM * kTiles - 1) / (kBM * kTiles), p.H, p.B);
-  attn_bf16_kernel<kSparse><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, prm);
+  // One CTA per SM: the items beyond the last whole wave form a partial
+  // wave.  If it fills at most half of the SMs, those items run split over
+  // KV halves (two CTAs each, a cluster per item) in a second launch.
+  int n_tail = 0;
+  if (!kSparse && n_kv >= 2) {
+    const int sms = device_sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    const int rem = static_cast<int>(n_items % sms);
+    if (2 * rem <= sms) n_tail = rem;
+  }
+  const int n_main = static_cast<int>(n_items) - n_tail;
+  if (n_main > 0) {
+    if ((e = set_smem_attr(reinterpret_cast<const void*>(attn_bf16_kernel<kSparse, false>), kSmemBytes)) !=
+        cudaSuccess)
+      return e;
+    attn_bf16_kernel<kSparse, false><<<n_main, kThreads, kSmemBytes, s>>>(tq, tk, tv, prm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if constexpr (!kSparse) {
+    if (n_tail > 0) {
+      const void* fn = reinterpret_cast<const void*>(attn_bf16_kernel<false, true>);
+      if ((e = set_smem_attr(fn, kSmemBytes)) != cudaSuccess) return e;
+      prm.item0 = n_main;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * n_tail, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      // Its CTAs may take SMs as the main launch's CTAs retire.
+      attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      if ((e = cudaLaunchKernelEx(&cfg, attn_bf16_kernel<false, true>, tq, tk, tv, prm)) != cudaSuccess) return e;
+    }
+  }
   return cudaGetLastError();
 }
 

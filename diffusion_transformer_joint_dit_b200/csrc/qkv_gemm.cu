@@ -72,6 +72,7 @@ struct Params {
   int k_steps;              // C / 64
   int tiles_txt, tiles_img; // 256-row tiles per batch element and stream
   int n_tiles_n;            // 3 H d / 256
+  int group_n;              // feature tiles per raster group
   int n_tiles;
   float eps;
   uint64_t timeout_ns;
@@ -81,11 +82,20 @@ struct Tile {
   int stream, b, tok0, tok_end, nt;
 };
 
+// Tile order: the feature tiles are cut into groups of group_n; group g
+// runs over every row tile before group g + 1 starts, row-major inside the
+// group.  The pairs working at one time then share a W panel set of group_n
+// feature tiles (sized on the host to stay resident in L2 while x streams
+// through), instead of needing all of W for every row tile.
 __device__ __forceinline__ Tile tile_at(const Params& p, int t) {
   Tile x;
-  x.nt = t % p.n_tiles_n;
-  const int mt = t / p.n_tiles_n;
   const int per_b = p.tiles_txt + p.tiles_img;
+  const int n_mt = p.B * per_b;
+  const int g = t / (n_mt * p.group_n);
+  const int width = min(p.group_n, p.n_tiles_n - g * p.group_n);
+  const int rg = t - g * n_mt * p.group_n;
+  const int mt = rg / width;
+  x.nt = g * p.group_n + (rg - mt * width);
   x.b = mt / per_b;
   const int r = mt - x.b * per_b;
   if (r < p.tiles_txt) {
@@ -304,7 +314,7 @@ qkv_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             uint4* dst = reinterpret_cast<uint4*>(orow + j * kD + c * 32);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4)
-              dst[q4] = make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
+              __stcs(dst + q4, make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]));
           }
         }
       }
@@ -351,6 +361,16 @@ cudaError_t launch_qkv_fused(const QkvProblem& q, cudaStream_t s) {
   p.tiles_txt = (q.n_txt + 2 * kBM - 1) / (2 * kBM);
   p.tiles_img = (q.N - q.n_txt + 2 * kBM - 1) / (2 * kBM);
   p.n_tiles_n = 3 * q.H * kD / kBN;
+  {
+    // Raster groups: the W panels of one group (kBN rows x C channels per
+    // feature tile, bf16) take at most 32 MiB, so that with the copies both
+    // halves of the L2 may hold they stay resident next to the x rows and
+    // the output lines in flight.
+    const long long panel = static_cast<long long>(kBN) * q.C * 2;
+    const long long budget = 32LL << 20;
+    const int n_groups = static_cast<int>((p.n_tiles_n * panel + budget - 1) / budget);
+    p.group_n = (p.n_tiles_n + n_groups - 1) / n_groups;
+  }
   const long long n_tiles = static_cast<long long>(q.B) * (p.tiles_txt + p.tiles_img) * p.n_tiles_n;
   if (n_tiles > 0x7fffffff) return cudaErrorInvalidValue;
   p.n_tiles = static_cast<int>(n_tiles);

@@ -157,6 +157,13 @@ JATTN_API int jattn_prologue(const void* q, const void* k, const void* v,
  * >= 1) but does not change the result: the sequence is attended as one.
  * d must be 128; softmax_scale must be finite and > 0.
  * o must not overlap q, k or v.
+ * Work items are 256 query rows of one (b, h), taken in (b, h, block)
+ * order, one per SM at a time.  When the items past the last whole wave
+ * fill at most half of the SMs (and N > 128), each of them runs as a
+ * cluster of two CTAs over the two halves of the keys, merged at the end;
+ * those rows differ from a one-pass computation by the merge's rounding
+ * only.  The result is deterministic: the same inputs on the same GPU give
+ * the same bits.
  */
 JATTN_API int jattn_fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse,
                    int B, int H, int N_txt, int N_img, int N_ref, int d,
