@@ -777,7 +777,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                       "attention_ms_median": att_med, "prologue_ms_median": pro_med,
                                       "attention_ms_plain_k": att_plain,
                                       "attention_tflops_plain_k": w.flops / (att_plain * 1e-3) / 1e12,
-                                      "prologue_gbs": 4 * act_bytes / (pro_ms * 1e-3) / 1e9}),
+                                      "prologue_gbs": 4 * act_bytes / (pro_ms * 1e-3) / 1e9,
+                                      # time x median SM clock of the timed region: compares runs
+                                      # taken in different power states
+                                      "attention_mcycles_at_median_clock":
+                                          att_ms * clocks["sm_mhz"] / 1e3 if (clocks or {}).get("sm_mhz")
+                                          else None}),
         "roofline": {
             "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "traffic": traffic,
