@@ -4,9 +4,9 @@ Inputs are the same bf16 tensors on both sides.  Small problems and the
 1024^2 workload are checked on every query row; the 2048^2 workloads run
 the kernel at full size in the benchmark's launch configuration and compare
 256 sampled query rows per (b, h) against all keys.  Tolerances: relative L2 <= 5e-3 and
-max-abs <= 2e-2 on the output; 2^-8 absolute on the log-sum-exp (the
-kernel sums the bf16-rounded P it multiplies V by, so ln l carries up to
-2^-9 relative rounding).
+max-abs <= 2e-2 on the output; 2^-8 absolute on the log-sum-exp (l counts
+each tile's largest P at its bf16 value, so ln l can carry up to 2^-9 of
+that term's rounding).
 """
 
 import numpy as np
@@ -49,6 +49,15 @@ def test_peaked_softmax_exercises_rescale(cuda_ok, gain):
     # Larger logits move the running max often (and by more than the lazy
     # rescale threshold), exercising the O correction path.
     _run(I.custom("peaked", B=1, H=2, n_txt=16, img_h=24, img_w=24), seed=11, q_gain=gain)
+
+
+@pytest.mark.parametrize("gain", [1.0, 12.0])
+def test_main_launch_and_split_tail_all_rows(cuda_ok, gain):
+    """162 work items on 148 SMs: a whole wave in the main launch and 14
+    items run split over KV halves (merged across a CTA pair), every row
+    checked; with gain 12 the two halves of a row keep different reference
+    maxima, which the merge has to reconcile."""
+    _run(I.custom("tail", B=1, H=9, n_txt=512, img_h=64, img_w=64), seed=31, q_gain=gain)
 
 
 def test_t2i_1024_all_rows(cuda_ok):

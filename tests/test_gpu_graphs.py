@@ -61,6 +61,24 @@ def test_bf16_step_in_a_graph(cuda_ok):
     _replay_matches(step, [q, k, v], [qo, ko, o, lse], seeds=[1, 2])
 
 
+def test_bf16_call_with_split_tail_in_a_graph(cuda_ok):
+    """A problem whose jattn_fwd_bf16 call is two launches on 148 SMs (162
+    work items: one whole wave, then 14 items run split over KV halves with
+    programmatic dependent launch) captured and replayed in a graph."""
+    w = I.custom("graph_tail", B=1, H=9, n_txt=512, img_h=64, img_w=64)
+    shape = (w.B, w.N, w.H, w.d)
+    q, k, v = (torch.empty(shape, dtype=torch.bfloat16, device="cuda") for _ in range(3))
+    o = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device="cuda")
+
+    def step():
+        J.jattn_fwd_bf16(q, k, v, o, lse, w.B, w.H, w.n_txt, w.n_img, w.n_ref, w.d, w.softmax_scale)
+
+    for t in (q, k, v):
+        t.normal_()
+    _replay_matches(step, [q, k, v], [o, lse], seeds=[3, 4])
+
+
 def test_fp8_step_with_repair_in_a_graph(cuda_ok):
     w = W
     shape = (w.B, w.N, w.H, w.d)
