@@ -257,8 +257,11 @@ repair_gather_kernel(const __grid_constant__ PrologueArgs a, const int* __restri
 //   O_c = W . V16       (kind::f16, A from TMEM)    -> TMEM [256, 384)
 // after which the thread rewrites its O and L rows.  With more than
 // kStageMax selected keys, the groups run one after another inside a pass,
-// accumulating O_c and z.  Exact K' and V rows must lie within the FP16
-// range (E4M3 codes and bf16 rows of moderate size are exact in FP16).
+// accumulating O_c and z.  With one group (the keys staged once) the passes
+// are pipelined: the next pass's S MMAs follow this pass's P.V in issue
+// order and run during its epilogue.  Exact K' and V rows must lie within
+// the FP16 range (E4M3 codes and bf16 rows of moderate size are exact in
+// FP16).
 constexpr int kApplyThreads = 128;
 constexpr int kApplyQ = 128;            // query rows per pass (= TMEM lanes)
 constexpr int kStageMax = 128;          // selected keys per group
@@ -443,6 +446,143 @@ repair_apply_kernel(const __grid_constant__ ApplyParams p) {
     lse_n = r < N ? p.lse[bh * N + r] : 0.f;
   };
   if (pass0 < pass1) prefetch(pass0 * kApplyQ);
+  if (ngroups == 1) {
+    // One key group, staged once: passes are pipelined.  The S MMAs of pass
+    // p + 1 are issued right after the P.V MMA of pass p (Q of pass p + 1
+    // is staged while W of pass p is formed), so they run during pass p's
+    // epilogue; S_x / S_q and W / O_c are separate TMEM regions.
+    const int ns = m, P = (m + 31) & ~31;
+    auto issue_s = [&]() {
+      tc_fence_after();
+      const uint32_t idesc_x = make_idesc(0, 0, false, kApplyQ, P);  // f16 x f16, K-major
+      const uint32_t idesc_q = make_idesc(0, 0, false, kApplyQ, P);  // e4m3 x e4m3, K-major
+      const uint32_t q16 = smem_u32(sm + kSmQ16), kx = smem_u32(sm + kSmKx);
+      const uint32_t q8 = smem_u32(sm + kSmQ8), kq = smem_u32(sm + kSmKq);
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk) {
+        const uint32_t aoff = (kk >> 2) * (kApplyQ * 128) + (kk & 3) * 32;
+        const uint32_t boff = (kk >> 2) * (P * 128) + (kk & 3) * 32;
+        mma_f16_ss(tmem + kColSx, smem_desc_sw128(q16 + aoff, 16, 1024), smem_desc_sw128(kx + boff, 16, 1024),
+                   idesc_x, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < kD / 32; ++kk)
+        mma_f8_ss(tmem + kColSq, smem_desc_sw128(q8 + kk * 32, 16, 1024), smem_desc_sw128(kq + kk * 32, 16, 1024),
+                  idesc_q, kk > 0 ? 1u : 0u);
+      mma_commit(&ctrl->s_full);
+    };
+    float cur_qsc = 0.f, cur_lse = 0.f;
+    if (pass0 < pass1) {
+      apply_store_q(sm, qn);
+      fence_proxy_async_smem();
+      cur_qsc = qsc_n;
+      cur_lse = lse_n;
+      if (pass0 + 1 < pass1) prefetch((pass0 + 1) * kApplyQ);
+      __syncthreads();
+      if (threadIdx.x == 0 && ok) issue_s();
+    }
+#pragma unroll 1
+    for (int pass = pass0; pass < pass1; ++pass) {
+      const int q0 = pass * kApplyQ;
+      const int row = q0 + threadIdx.x;
+      const bool live = row < N;
+      const float lse_row = cur_lse;
+      const float l2 = lse_row * log2e;
+      const float sx = cur_qsc * p.scale_log2;
+      float z = 0.f;
+      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * N + (live ? row : 0)) * p.H + h) * kD;
+      if (ok) ok = mbar_wait(&ctrl->s_full, s_phase & 1u, abort_flag, p.timeout_ns);
+      ++s_phase;
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < P; c0 += 32) {
+          uint32_t ax[32], aq[32];
+          tmem_ld32(tmem + lane_sel + kColSx + c0, ax);
+          tmem_ld32(tmem + lane_sel + kColSq + c0, aq);
+          tmem_ld_wait(ax);
+          tmem_ld_wait(aq);
+          uint32_t wx[16], wq[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float ex[2], eq[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int key = c0 + j + u;
+              const bool in = key < ns;
+              ex[u] = in ? ex2_approx(__uint_as_float(ax[j + u]) * sx - l2) : 0.f;
+              eq[u] = in ? ex2_approx(__uint_as_float(aq[j + u]) * (sx * s_ks[key]) - l2) : 0.f;
+              z += ex[u] - eq[u];
+              eq[u] *= -s_vs[key];  // V's block scale folded into the weight of the codes
+            }
+            wx[j >> 1] = pack_f16x2(ex[0], ex[1]);
+            wq[j >> 1] = pack_f16x2(eq[0], eq[1]);
+          }
+          tmem_st16(tmem + lane_sel + kColW + c0 / 2, wx);
+          tmem_st16(tmem + lane_sel + kColW + P / 2 + c0 / 2, wq);
+        }
+        tmem_st_wait();
+      }
+      // The S MMAs of this pass have completed: the Q buffer takes the next
+      // pass's rows.
+      float nxt_qsc = 0.f, nxt_lse = 0.f;
+      if (pass + 1 < pass1) {
+        apply_store_q(sm, qn);
+        fence_proxy_async_smem();
+        nxt_qsc = qsc_n;
+        nxt_lse = lse_n;
+      }
+      tc_fence_before();
+      __syncthreads();  // W of every row in TMEM, S read, next Q staged
+      if (threadIdx.x == 0 && ok) {
+        tc_fence_after();
+        const uint32_t v16 = smem_u32(sm + kSmV);
+#pragma unroll 1
+        for (int kk = 0; kk < (2 * P) / 16; ++kk)
+          mma_f16_ts(tmem + kColO, tmem + kColW + kk * 8, smem_desc_sw128(v16 + kk * 16 * 128, 2 * P * 128, 1024),
+                     idesc_pv, kk > 0 ? 1u : 0u);
+        mma_commit(&ctrl->o_full);
+        if (pass + 1 < pass1) issue_s();  // in issue order after P.V, which read W
+      }
+      if (pass + 2 < pass1) prefetch((pass + 2) * kApplyQ);  // in flight during the epilogue
+      uint4 o_in[kD / 8];
+#pragma unroll
+      for (int i = 0; i < kD / 8; ++i)
+        o_in[i] = live ? *reinterpret_cast<const uint4*>(orow + i * 8) : make_uint4(0, 0, 0, 0);
+      if (ok) ok = mbar_wait(&ctrl->o_full, o_phase & 1u, abort_flag, p.timeout_ns);
+      ++o_phase;
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        const float inv = 1.f / (1.f + z);
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_sel + kColO + c * 32, a);
+          tmem_ld_wait(a);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 ov = o_in[c * 4 + q4];
+            const uint32_t w[4] = {ov.x, ov.y, ov.z, ov.w};
+            uint32_t r[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float lo = (__uint_as_float(w[i] << 16) + __uint_as_float(a[q4 * 8 + 2 * i])) * inv;
+              const float hi = (__uint_as_float(w[i] & 0xFFFF0000u) + __uint_as_float(a[q4 * 8 + 2 * i + 1])) * inv;
+              r[i] = pack_bf16x2(lo, hi);
+            }
+            if (live) *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = make_uint4(r[0], r[1], r[2], r[3]);
+          }
+        }
+        if (live) p.lse[bh * N + row] = lse_row + __logf(1.f + z);
+      }
+      tc_fence_before();
+      __syncthreads();  // O_c read before the next pass's P.V overwrites it
+      cur_qsc = nxt_qsc;
+      cur_lse = nxt_lse;
+    }
+  } else
 #pragma unroll 1
   for (int pass = pass0; pass < pass1; ++pass) {
     const int q0 = pass * kApplyQ;
