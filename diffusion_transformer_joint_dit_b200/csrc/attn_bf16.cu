@@ -48,7 +48,9 @@
 // CTA 0 merges the two halves:
 //   m = max(m0, m1),  l = 2^(m0-m) l0 + 2^(m1-m) l1,
 //   O = (2^(m0-m) O0 + 2^(m1-m) O1) / l.
-// The partial wave then takes half as long.
+// The partial wave then takes half as long.  After a main launch the tail
+// uses programmatic dependent launch (its CTAs take SMs as the main
+// launch's retire) and completes only after the main launch has.
 //
 // Block-sparse variant (kSparse): the tutorial's Sol-Attention runs a
 // generic block-sparse attention kernel.  A CTA's 256 query rows are one
@@ -564,11 +566,16 @@ cudaError_t launch_bf16(const AttnProblem& p, const int* kv_idx, const int* kv_c
       attr[0].val.clusterDim.x = 2;
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
-      // Its CTAs may take SMs as the main launch's CTAs retire.
+      // After a main launch, the tail's CTAs may take SMs as the main
+      // launch's CTAs retire: the main kernel releases them at its start,
+      // and the tail reads nothing the main launch writes (the inputs were
+      // complete before the main launch began).  Without a main launch the
+      // tail is ordered normally after whatever precedes it, whose results
+      // it reads.
       attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
       attr[1].val.programmaticStreamSerializationAllowed = 1;
       cfg.attrs = attr;
-      cfg.numAttrs = 2;
+      cfg.numAttrs = n_main > 0 ? 2 : 1;
       if ((e = cudaLaunchKernelEx(&cfg, attn_bf16_kernel<false, true>, tq, tk, tv, prm)) != cudaSuccess) return e;
     }
   }
